@@ -1,0 +1,493 @@
+"""Pins of the CPU oracle to what the pages and the mathematics fix (no GPU).
+
+Every test compares the oracle with something other than itself: values the pages print
+(tests/golden/), exhaustive nearest-value searches in exact rationals (tests/exact.py),
+closed forms, invariants, special cases, and library routines (torch's CPU casts).
+"""
+from __future__ import annotations
+
+import math
+import os
+import struct
+from fractions import Fraction as F
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from tests import exact as X
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def golden_rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.split("#")[0].strip() for ln in f if ln.split("#")[0].strip()]
+
+
+def f32(v) -> float:
+    return struct.unpack("<f", struct.pack("<f", float(v)))[0]
+
+
+def bits_to_f32(u: int) -> float:
+    return struct.unpack("<f", struct.pack("<I", u & 0xFFFFFFFF))[0]
+
+
+def bf16_bits(vals) -> np.ndarray:
+    return torch.tensor(vals, dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_exact(vals) -> np.ndarray:
+    b = bf16_bits(vals)
+    back = torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).float().numpy()
+    assert np.array_equal(back, np.asarray(vals, np.float32)), "fixture value not exact in BF16"
+    return b
+
+
+# ---- P1: the E2M1 grid -------------------------------------------------------------------
+
+def test_p1_e2m1_grid_matches_pages():
+    rows = [r.split() for r in golden_rows("e2m1_grid.txt")]
+    for idx, val in rows:
+        assert O.e2m1_to_f32([int(idx)])[0] == float(val)
+        neg = O.e2m1_to_f32([int(idx) | 8])[0]
+        assert neg == -float(val) and math.copysign(1.0, neg) == -1.0
+
+
+def test_p2_step_sizes():
+    mags = O.e2m1_to_f32(range(8))
+    steps = np.diff(mags)
+    assert list(steps[:4]) == [0.5] * 4          # 0 .. 2
+    assert list(steps[4:6]) == [1.0, 1.0]        # 2 .. 4
+    assert list(steps[6:]) == [2.0]              # 4 .. 6
+
+
+# ---- P2/P5: rounding of scaled values ----------------------------------------------------
+
+def test_p2_rounding_table_from_pages():
+    for row in golden_rows("e2m1_rounding.txt"):
+        parts = row.split()
+        y, want = float(parts[0]), float(parts[1])
+        got = O.e2m1_to_f32(O.f32_to_e2m1([y]))[0]
+        assert got == want, (y, got, want)
+        gotn = O.e2m1_to_f32(O.f32_to_e2m1([-y]))[0]
+        assert gotn == -want and math.copysign(1.0, gotn) == -1.0
+
+
+def test_p5_five_goes_to_four_or_six():
+    five = f32(5.0)
+    up = np.nextafter(np.float32(5.0), np.float32(10.0))
+    down = np.nextafter(np.float32(5.0), np.float32(0.0))
+    assert O.e2m1_to_f32(O.f32_to_e2m1([five]))[0] == 4.0
+    assert O.e2m1_to_f32(O.f32_to_e2m1([up]))[0] == 6.0
+    assert O.e2m1_to_f32(O.f32_to_e2m1([down]))[0] == 4.0
+
+
+def _e2m1_probe_values():
+    rng = np.random.default_rng(123)
+    vals = set()
+    # every midpoint and grid point, +-8 ulps
+    for p in [0, 0.25, 0.5, 0.75, 1, 1.25, 1.5, 1.75, 2, 2.5, 3, 3.5, 4, 5, 6, 7, 8]:
+        b = struct.unpack("<I", struct.pack("<f", p))[0]
+        for k in range(-8, 9):
+            if p == 0 and k < 0:
+                continue
+            vals.add(bits_to_f32(b + k))
+    # a sweep of the range and far beyond, plus subnormals and huge values
+    vals.update(float(v) for v in rng.uniform(0, 8, 4000).astype(np.float32))
+    vals.update(float(v) for v in np.exp2(rng.uniform(-149, 127, 2000)).astype(np.float32))
+    vals.update([bits_to_f32(1), bits_to_f32(0x7F7FFFFF), float("inf")])
+    return sorted(vals)
+
+
+def test_p2_e2m1_exhaustive_nearest_in_exact_rationals():
+    """Brute force: the code of y is the grid value nearest to y (exact distances), ties to
+    the even code, values beyond 6 saturate to 6; the sign bit follows y's sign bit."""
+    vals = _e2m1_probe_values()
+    got = O.f32_to_e2m1(vals + [-v for v in vals])
+    n = len(vals)
+    for i, y in enumerate(vals):
+        if math.isinf(y):
+            want = 7
+        else:
+            want, _ = X.nearest_ties_even(X.f32_value(y), X.E2M1_GRID)
+        assert got[i] == want, (y, got[i], want)
+        assert got[n + i] == (want | 8), (-y, got[n + i])
+
+
+# ---- E4M3 and BF16 conversions against definitions and library routines ---------------------
+
+def test_p10_e4m3_decode_all_codes_against_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy()
+    got = O.e4m3_to_f32(codes)
+    finite = ~np.isnan(ref)
+    assert np.array_equal(got[finite], ref[finite])
+    assert np.all(np.isnan(got[~finite]))
+    assert list(np.where(~finite)[0]) == [0x7F, 0xFF]
+
+
+def test_p10_e4m3_encode_against_torch_in_range():
+    """In range (|t| <= 448) torch's CPU cast rounds to nearest even, like the oracle."""
+    rng = np.random.default_rng(7)
+    t = np.concatenate([
+        np.exp2(rng.uniform(-12, np.log2(448.0), 20000)),
+        rng.uniform(0, 448, 5000),
+        torch.arange(0, 0x43E0, dtype=torch.int16).view(torch.bfloat16).float().numpy(),  # every BF16 <= 448
+    ]).astype(np.float32)
+    t = t[t <= 448.0]
+    # exact ties between neighbouring E4M3 values
+    vals = X.E4M3
+    ties = np.array([float((vals[k] + vals[k + 1]) / 2) for k in range(len(vals) - 1)], np.float32)
+    t = np.concatenate([t, ties, -t])
+    ref = torch.from_numpy(t).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = O.f32_to_e4m3(t)
+    assert np.array_equal(got, ref)
+
+
+def test_p10_e4m3_saturates_at_448():
+    for t in [448.0, 449.0, 463.9, 464.0, 464.1, 480.0, 1e6, 3.0e38, float("inf")]:
+        assert O.f32_to_e4m3([t])[0] == 0x7E
+        assert O.f32_to_e4m3([-t])[0] == 0xFE
+
+
+def test_e4m3_exhaustive_nearest_in_exact_rationals():
+    rng = np.random.default_rng(11)
+    probes = set(float(v) for v in np.exp2(rng.uniform(-14, 10, 3000)).astype(np.float32))
+    for k in range(len(X.E4M3) - 1):
+        mid = (X.E4M3[k] + X.E4M3[k + 1]) / 2
+        b = struct.unpack("<I", struct.pack("<f", float(mid)))[0]
+        for d in (-2, -1, 0, 1, 2):
+            probes.add(bits_to_f32(b + d))
+    probes = sorted(probes)
+    got = O.f32_to_e4m3(probes)
+    for t, g in zip(probes, got):
+        want, _ = X.nearest_ties_even(X.f32_value(t), X.E4M3)
+        assert g == want, (t, g, want)
+
+
+def test_bf16_rounding_against_torch():
+    rng = np.random.default_rng(5)
+    u = rng.integers(0, 2**32, 200000, dtype=np.uint64).astype(np.uint32)
+    f = u.view(np.float32)
+    f = f[np.isfinite(f)]
+    # exact ties (low half exactly 0x8000) and the overflow boundary
+    ties = ((rng.integers(0, 2**16, 5000, dtype=np.uint32) << 16) | 0x8000).view(np.float32)
+    edge = np.array([3.3895314e38, 3.3961776e38, 3.4028235e38, -3.40282e38, 1e-45, -1e-45, 0.0, -0.0],
+                    np.float32)
+    f = np.concatenate([f, ties[np.isfinite(ties)], edge])
+    ref = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = O.f32_to_bf16(f)
+    assert np.array_equal(got, ref)
+
+
+# ---- P14: amax -----------------------------------------------------------------------------
+
+def test_p14_amax_against_torch():
+    from nvfp4_block_scaled_13_b200 import synth
+
+    for name, rows, cols, groups in [("c3", 8, 256, 1), ("c4", 16, 64, 5), ("c5", 64, 128, 1)]:
+        x, (g, r, c) = synth.make(name, rows=rows, cols=cols, groups=groups)
+        got = O.amax(x, g, r, c)
+        t = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).float().reshape(g, -1)
+        ref = t.abs().amax(dim=1).numpy()
+        assert np.array_equal(got, ref)
+
+
+# ---- P3 / P4 / P6: worked blocks from the pages --------------------------------------------
+
+def _parse_worked():
+    out = []
+    for row in golden_rows("worked_blocks.txt"):
+        head, xs, sc, qs, ch = [p.strip() for p in row.split("|")]
+        name, mode, rule, amax = head.split()
+        out.append(dict(name=name, mode=int(mode), rule=int(rule), amax=float(amax),
+                        x=[float(v) for v in xs.split()], scale=int(sc, 16),
+                        q=[float(v) for v in qs.split()], choice=int(ch)))
+    return out
+
+
+@pytest.mark.parametrize("case", _parse_worked(), ids=lambda c: f"{c['name']}-r{c['rule']}")
+def test_p3_p4_worked_blocks(case):
+    x = bf16_exact(case["x"])
+    o = O.quantize(x, 1, 1, 16, np.array([case["amax"]], np.float32), case["mode"], case["rule"])
+    assert o["scales"][0] == case["scale"]
+    assert o["tscale"][0] == 1.0
+    assert int(o["choice"][0]) & 1 == case["choice"]
+    fq = O.fakequant(x, 1, 1, 16, np.array([case["amax"]], np.float32), case["mode"], case["rule"])["fq"]
+    want = bf16_exact(case["q"])
+    assert np.array_equal(fq, want), (fq, want)
+
+
+def test_p3_near_max_values_only_reach_4_or_6():
+    """Scale-6 block with maximum m: every value in (2/3 m, m) dequantizes to 4d or 6d."""
+    m = 2688.0
+    vals = torch.arange(1792, 2688, 16, dtype=torch.float32)  # every BF16 value in [2/3 m, m)
+    for start in range(0, len(vals), 15):
+        chunk = [m] + vals[start:start + 15].tolist()
+        chunk += [0.0] * (16 - len(chunk))
+        x = bf16_exact(chunk)
+        fq = O.fakequant(x, 1, 1, 16, np.array([m], np.float32), O.SCALE6, O.RULE_MSE)["fq"]
+        back = torch.from_numpy(fq.view(np.int16)).view(torch.bfloat16).float().numpy()
+        for v, q in zip(chunk[1:], back[1:]):
+            if v > 0:
+                assert q in (1792.0, 2688.0), (v, q)
+        assert fq[0] == bf16_exact([m])[0]
+
+
+def test_p4_three_quarters_lands_on_three():
+    c4 = O.block_candidate([1536.0, 1152.0] + [0.0] * 14, 1.0, 4.0, O.RULE_MSE)
+    assert c4.s == 0x7C and c4.d == 384.0
+    assert (c4.code[1] & 7) == 5 and c4.e[1] == 0.0          # 0.75 * max -> 3 exactly
+    c6 = O.block_candidate([1536.0, 1152.0] + [0.0] * 14, 1.0, 6.0, O.RULE_MSE)
+    assert c6.s == 0x78 and c6.d == 256.0
+    assert (c6.code[1] & 7) == 6 and c6.e[1] == 128.0        # 4.5 -> 4, error d6 / 2
+
+
+def test_p6_zero_blocks_and_zero_groups():
+    # an all-zero group (amax 0): alpha 0, scale 0, codes keep the sign, choice 6, output +-0
+    x = bf16_exact([0.0, -0.0] * 8)
+    for mode in (O.SCALE6, O.FOUR_OVER_SIX):
+        for rule in (O.RULE_MAXERR, O.RULE_MAE, O.RULE_MSE):
+            o = O.quantize(x, 1, 1, 16, np.zeros(1, np.float32), mode, rule)
+            assert o["tscale"][0] == 0.0 and o["scales"][0] == 0 and o["choice"][0] == 0
+            assert list(o["codes"]) == [0x80] * 8
+            fq = O.fakequant(x, 1, 1, 16, np.zeros(1, np.float32), mode, rule)["fq"]
+            assert np.array_equal(fq, x)
+    # a zero block inside a non-zero tensor
+    x = bf16_exact([3.0] * 16 + [0.0] * 8 + [-0.0] * 8)
+    o = O.quantize(x, 1, 1, 32, np.array([3.0], np.float32), O.FOUR_OVER_SIX, O.RULE_MSE)
+    assert o["scales"][1] == 0 and list(o["codes"][8:]) == [0] * 4 + [0x88] * 4
+    assert (o["choice"][0] >> 1) & 1 == 0
+
+
+# ---- layout -----------------------------------------------------------------------------------
+
+def test_layout_example():
+    rows = {r.split(":")[0]: r.split(":")[1].split() for r in golden_rows("layout_example.txt")}
+    x = bf16_exact([float(v) for v in rows["x"]])
+    o = O.quantize(x, 1, 1, 32, np.array([1536.0], np.float32), O.FOUR_OVER_SIX, O.RULE_MSE)
+    assert list(o["codes"]) == [int(v, 16) for v in rows["codes"]]
+    assert list(o["scales"]) == [int(v, 16) for v in rows["scales"]]
+    assert o["tscale"][0] == float(rows["tscale"][0])
+    assert list(o["choice"]) == [int(v, 16) for v in rows["choice"]]
+    y = O.dequantize(o["codes"], o["scales"], o["tscale"], 1, 1, 32)
+    assert np.array_equal(y, bf16_exact([float(v) for v in rows["dequantized"]]))
+
+
+# ---- P7: brute force of the whole block pipeline in exact rationals ---------------------------
+
+def _exact_candidate(xs, amax, M, K, rule):
+    """Exact-arithmetic version of one candidate plus error bounds on the oracle's binary32
+    path (u = 2^-24 per rounding). Returns None where a decision is too close to call."""
+    u = X.U
+    alpha = F(amax) / (6 * M)
+    m = max(abs(v) for v in xs)
+    # relative error bound on t = m / (K alpha) as the oracle computes it
+    ex_alpha = X.is_f32(alpha)
+    beta = K * alpha
+    t = m / beta if beta > 0 else F(0)
+    exact_t = ex_alpha and X.is_f32(beta) and X.is_f32(t)
+    dt = F(0) if exact_t else 4 * u
+    s_idx, margin = X.nearest_ties_even(t, X.E4M3)
+    if dt > 0 and margin <= dt * t * F(101, 100):
+        return None
+    s = X.E4M3[s_idx]
+    d = s * alpha
+    exact_d = ex_alpha and X.is_f32(d)
+    dd = F(0) if exact_d else 2 * u
+    exact_r = exact_d and d > 0 and X.is_f32(1 / d)
+    dr = F(0) if exact_r else dd + u
+    codes, errs, bounds, qs = [], [], [], []
+    for v in xs:
+        if d == 0:
+            y = F(0)
+            exact_y = True
+        else:
+            y = v / d
+            exact_y = exact_r and X.is_f32(v * (1 / d))
+        dy = F(0) if exact_y else dr + u
+        idx, mg = X.nearest_ties_even(abs(y), X.E2M1_GRID)
+        if dy > 0 and mg <= dy * abs(y) * F(101, 100) and abs(y) < 6:
+            return None
+        val = X.E2M1_GRID[idx] * (1 if v >= 0 else -1)
+        q = val * d
+        e = v - q
+        exact_e = exact_y and X.is_f32(q) and X.is_f32(e)
+        b = F(0) if exact_e else (abs(q) * (dd + u) + abs(e) * u) * F(102, 100)
+        codes.append(idx)
+        errs.append(e)
+        bounds.append(b)
+        qs.append(q)
+    if rule == 0:
+        err = max(abs(e) for e in errs)
+        bound = max(bounds)
+    elif rule == 1:
+        err = sum(abs(e) for e in errs)
+        all_exact = all(b == 0 for b in bounds) and all(X.is_f32(sum(abs(e) for e in errs[p::2][:k]))
+                                                        for p in (0, 1) for k in range(1, 9))
+        bound = F(0) if all_exact and X.is_f32(err) else sum(bounds) + 17 * u * err
+    else:
+        err = sum(e * e for e in errs)
+        all_exact = all(b == 0 for b in bounds) and all(X.is_f32(e * e) for e in errs) and \
+            all(X.is_f32(sum(e * e for e in errs[p::2][:k])) for p in (0, 1) for k in range(1, 9))
+        bound = F(0) if all_exact and X.is_f32(err) else \
+            sum(2 * abs(e) * b + b * b for e, b in zip(errs, bounds)) + 18 * u * err
+    return dict(s=s_idx, codes=codes, err=err, bound=bound, q=qs)
+
+
+def _lattice_blocks(rng, n):
+    """Blocks of small-lattice BF16 values (many exact ties under power-of-two scales)."""
+    out = []
+    for _ in range(n):
+        scale = F(2) ** int(rng.integers(-6, 7))
+        k = rng.integers(-47, 48, 16)
+        if rng.random() < 0.5:
+            k[int(rng.integers(0, 16))] = 48 * (1 if rng.random() < 0.5 else -1)   # max 6 * scale
+        vals = [F(int(v)) / 8 * scale for v in k]
+        if rng.random() < 0.3:
+            vals[int(rng.integers(0, 16))] = F(0)
+        out.append(vals)
+    return out
+
+
+@pytest.mark.parametrize("mode,rule", [(0, 2), (1, 0), (1, 1), (1, 2)])
+def test_p7_block_pipeline_brute_force_exact(mode, rule):
+    rng = np.random.default_rng(1000 + 10 * mode + rule)
+    M = 256 if mode == 1 else 448
+    blocks = _lattice_blocks(rng, 320)
+    checked = ties = near = 0
+    for vals in blocks:
+        m = max(abs(v) for v in vals)
+        if m == 0:
+            continue
+        # amax: the block max itself, a power-of-two multiple of 6M (alpha exact), or a
+        # random larger value (alpha inexact)
+        pick = int(rng.integers(0, 3))
+        if pick == 0:
+            amax = m
+        elif pick == 1:
+            amax = 6 * M * F(2) ** int(math.ceil(math.log2(float(m) / (6 * M))))
+        else:
+            amax = m * F(int(rng.integers(100, 400)), 100)
+        amax_f = f32(float(amax))
+        amax = X.f32_value(amax_f)
+        x = bf16_exact([float(v) for v in vals])
+        o = O.quantize(x, 1, 1, 16, np.array([amax_f], np.float32), mode, rule)
+        codes = [(int(o["codes"][j // 2]) >> (4 * (j % 2))) & 0xF for j in range(16)]
+        c6 = _exact_candidate(vals, amax, M, 6, rule)
+        c4 = _exact_candidate(vals, amax, M, 4, rule) if mode == 1 else None
+        if c6 is None or (mode == 1 and c4 is None):
+            near += 1
+            continue
+        if mode == 0:
+            pick4 = False
+        else:
+            gap = abs(c4["err"] - c6["err"])
+            if gap == 0 and c4["bound"] == 0 and c6["bound"] == 0:
+                pick4 = False          # exact tie keeps target 6
+                ties += 1
+            elif gap > c4["bound"] + c6["bound"]:
+                pick4 = c4["err"] < c6["err"]
+            else:
+                near += 1
+                continue
+        want = c4 if pick4 else c6
+        assert int(o["choice"][0]) & 1 == int(pick4), (vals, amax)
+        assert o["scales"][0] == want["s"], (vals, amax, o["scales"][0], want["s"])
+        assert [c & 7 for c in codes] == want["codes"], (vals, amax, codes, want["codes"])
+        assert [c >> 3 for c in codes] == [1 if v < 0 else 0 for v in vals]
+        checked += 1
+    assert checked >= 150, (checked, near, ties)
+
+
+# ---- P8: invariants of the choice -------------------------------------------------------------
+
+@pytest.mark.parametrize("rule", [0, 1, 2])
+def test_p8_chosen_error_not_larger(rule):
+    from nvfp4_block_scaled_13_b200 import synth
+
+    x, (g, r, c) = synth.make("c3", rows=8, cols=256)
+    xf = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).float().numpy().reshape(-1, 16)
+    amax = O.amax(x, g, r, c)
+    alpha = O.tensor_scale(amax[0], O.FOUR_OVER_SIX)
+    o = O.quantize(x, g, r, c, amax, O.FOUR_OVER_SIX, rule)
+    for b in range(xf.shape[0]):
+        c6 = O.block_candidate(xf[b], alpha, 6.0, rule)
+        c4 = O.block_candidate(xf[b], alpha, 4.0, rule)
+        chosen4 = (o["choice"][b // 8] >> (b % 8)) & 1
+        err_chosen = c4.err if chosen4 else c6.err
+        assert err_chosen <= min(c4.err, c6.err)
+        assert o["scales"][b] == (c4.s if chosen4 else c6.s)
+
+
+# ---- P9: tensor-scale invariants (256 vs 448) -------------------------------------------------
+
+def test_p9_amax_block_scales():
+    from nvfp4_block_scaled_13_b200 import synth
+
+    for name in ("c1", "c2", "c3"):
+        x, (g, r, c) = synth.make(name, rows=16, cols=256)
+        xf = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).float().numpy()
+        amax = O.amax(x, g, r, c)
+        top = int(np.argmax(np.abs(xf))) // 16
+        o6 = O.quantize(x, g, r, c, amax, O.SCALE6, O.RULE_MSE)
+        assert o6["scales"][top] == 0x7E                     # 448
+        o4 = O.quantize_ex(x, g, r, c, amax, 256.0, 2, O.RULE_MSE)
+        o6b = O.quantize_ex(x, g, r, c, amax, 256.0, 1, O.RULE_MSE)
+        assert o6b["scales"][top] == 0x78 and o4["scales"][top] == 0x7C   # 256 and 384 = 1.5 x 256
+        assert o4["scales"].max() <= 0x7C                   # target-4 scales never saturate
+        # built from 448 instead, the target-4 scale of the top block would need 672: it clips
+        o4_448 = O.quantize_ex(x, g, r, c, amax, 448.0, 2, O.RULE_MSE)
+        assert o4_448["scales"][top] == 0x7E
+
+
+# ---- P11 / P12 / P13 ------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode,rule", [(0, 2), (1, 0), (1, 1), (1, 2)])
+def test_p11_dequantize_of_quantize_equals_fakequant(mode, rule):
+    from nvfp4_block_scaled_13_b200 import synth
+
+    x, (g, r, c) = synth.make("c4", rows=8, cols=64, groups=3)
+    amax = O.amax(x, g, r, c)
+    o = O.quantize(x, g, r, c, amax, mode, rule)
+    fq = O.fakequant(x, g, r, c, amax, mode, rule)
+    assert np.array_equal(O.dequantize(o["codes"], o["scales"], o["tscale"], g, r, c), fq["fq"])
+    assert np.array_equal(o["choice"], fq["choice"])
+
+
+def test_p12_storage_closed_form():
+    g, r, c = 1, 64, 1024
+    n = g * r * c
+    o = O.quantize(np.zeros(n, np.uint16), g, r, c, np.zeros(1, np.float32), 1, 2)
+    bits = 8 * (o["codes"].nbytes + o["scales"].nbytes)
+    assert bits / n == 4.5
+    assert o["choice"].nbytes == n // 128
+    assert math.isclose(16 / 4.5, 3.5556, rel_tol=1e-4)      # vs BF16
+    assert math.isclose(8 / 4.5, 1.7778, rel_tol=1e-4)       # vs FP8 (pages: "1.7x")
+
+
+@pytest.mark.parametrize("rule", [0, 1, 2])
+def test_p13_four_over_six_reduces_to_single_candidate_runs(rule):
+    from nvfp4_block_scaled_13_b200 import synth
+
+    x, (g, r, c) = synth.make("c2", rows=32, cols=256)
+    amax = O.amax(x, g, r, c)
+    both = O.quantize(x, g, r, c, amax, O.FOUR_OVER_SIX, rule)
+    only6 = O.quantize_ex(x, g, r, c, amax, 256.0, 1, rule)
+    only4 = O.quantize_ex(x, g, r, c, amax, 256.0, 2, rule)
+    nb = g * r * c // 16
+    bits = np.unpackbits(both["choice"], bitorder="little")[:nb].astype(bool)
+    assert 0 < bits.sum() < nb
+    assert np.array_equal(both["scales"][~bits], only6["scales"][~bits])
+    assert np.array_equal(both["scales"][bits], only4["scales"][bits])
+    cb = both["codes"].reshape(nb, 8)
+    assert np.array_equal(cb[~bits], only6["codes"].reshape(nb, 8)[~bits])
+    assert np.array_equal(cb[bits], only4["codes"].reshape(nb, 8)[bits])
+    # standard scale-6 mode is the target-6-only run with the tensor scale built from 448
+    s6 = O.quantize(x, g, r, c, amax, O.SCALE6, rule)
+    s6b = O.quantize_ex(x, g, r, c, amax, 448.0, 1, rule)
+    for k in ("codes", "scales", "tscale", "choice"):
+        assert np.array_equal(s6[k], s6b[k])
+    assert not s6["choice"].any()
