@@ -1,0 +1,151 @@
+/*
+ * nvfp4.h — C ABI of libnvfp4.so: BF16 -> NVFP4 block-scaled quantization on NVIDIA B200
+ * (sm_100a), with standard "scale-6" blocks and Four Over Six adaptive block scaling.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [FOS] "Four Over Six: More Accurate NVFP4 Quantization with Adaptive Block Scaling"
+ *         (gist.science explainer), technical summary: Problem definition; Method > Core
+ *         mechanism; Method > Adaptive block scaling algorithm; Implementation details.
+ *   [QAD] "Quantization-Aware Distillation for NVFP4 Inference Accuracy Recovery"
+ *         (gist.science explainer), technical summary §3.3: NVFP4 blocks of 16 values.
+ *   [N35] "NVIDIA、「Nemotron 3.5 Lightning」のNVFP4量子化手法を公開" (news article), two-stage
+ *         QAD section: the student's forward pass runs through simulated quantization.
+ *
+ * The number format. A tensor x of BF16 values, viewed as [groups, rows, cols] row-major, is
+ * cut into blocks of 16 consecutive elements along the last dimension ([QAD] §3.3). Each
+ * group g has an FP32 tensor scale alpha_g; each block b has an FP8 E4M3 scale s_b; each
+ * element is a 4-bit E2M1 code c (sign bit 3, magnitude index bits 0-2 into the grid
+ * {0, 0.5, 1, 1.5, 2, 3, 4, 6}, [FOS] Problem definition). The stored value is
+ *     v(c) * s_b * alpha_g.
+ *
+ * The computation (every operation IEEE binary32, round to nearest even):
+ *     alpha  = amax_g / (6 * M),  M = 448 in scale-6 mode, 256 in Four Over Six mode
+ *              ([FOS] Implementation details: 256 instead of 448 leaves room for the 1.5x
+ *              larger scale of a target-4 block)
+ *     for each candidate target maximum K (scale-6 mode: K = 6; Four Over Six: K = 6 and 4,
+ *     [FOS] Core mechanism and Adaptive block scaling algorithm: quantize twice):
+ *       beta = K * alpha;  t = m_b / beta (0 if beta <= 0), m_b = max |x| over the block
+ *       s    = E4M3(t), round to nearest even, saturating at 448
+ *       d    = f32(s) * alpha;  r = (d > 0) ? min(1 / d, FLT_MAX) : 0
+ *       c_i  = E2M1(x_i * r), round to nearest even, saturating at 6, sign kept
+ *       q_i  = v(c_i) * d;  e_i = x_i - q_i   (error against the original values)
+ *       err  = MAXERR: max |e_i|;  MAE: S(|e_i|);  MSE: S(e_i^2) with fused multiply-add,
+ *              where S sums even-indexed and odd-indexed terms in two running sums (each in
+ *              increasing index order, starting from +0) and then adds the two
+ *     Four Over Six keeps target 4 iff err_4 < err_6 (ties keep 6, the standard format),
+ *     under one of the three rules of [FOS] Adaptive block scaling algorithm.
+ * Results are bit-identical to the CPU oracle that ships with the tests.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller. The library allocates no
+ *     memory, keeps no state between calls and never synchronizes the host: work is enqueued
+ *     on `stream` (0 = the legacy default stream) and completes in stream order.
+ *   - Shapes: groups >= 1, rows >= 0, cols >= 0 with cols % 16 == 0. An empty tensor
+ *     (rows == 0 or cols == 0) is valid; each function states what it writes for one.
+ *   - Alignment: BF16 tensors (x, y) 32 bytes, codes 8 bytes, choice/amax/tscale 4 bytes.
+ *     Memory from cudaMalloc or torch satisfies all of these.
+ *   - Inputs must be finite and amax values finite and >= 0; NaN/Inf inputs do not fault but
+ *     give unspecified outputs. Output buffers must not overlap inputs or each other.
+ *   - Errors: argument errors are detected on the host and returned before anything is
+ *     enqueued (no output is touched). A launch failure returns NVFP4_ERR_CUDA. Kernels
+ *     contain no device-side assert, trap or wait.
+ *   - Buffers must live on the device that is current for the calling thread.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_NULL = 1,    /* a required pointer is NULL                                 */
+    NVFP4_ERR_SHAPE = 2,   /* groups < 1, negative rows/cols, cols % 16 != 0, or overflow */
+    NVFP4_ERR_ALIGN = 3,   /* a pointer violates the alignment rule above                 */
+    NVFP4_ERR_MODE = 4,    /* unknown nvfp4_mode                                          */
+    NVFP4_ERR_RULE = 5,    /* unknown nvfp4_rule (checked in Four Over Six mode only)     */
+    NVFP4_ERR_CUDA = 6     /* the CUDA runtime reported an error while enqueuing          */
+} nvfp4_status;
+
+/* Block-scale selection ([FOS] Problem definition; Core mechanism). */
+typedef enum {
+    NVFP4_SCALE6 = 0,          /* standard NVFP4: every block's maximum maps to 6, M = 448 */
+    NVFP4_FOUR_OVER_SIX = 1    /* per block, the better of max 6 and max 4, M = 256        */
+} nvfp4_mode;
+
+/* Error rule for Four Over Six ([FOS] Adaptive block scaling algorithm). */
+typedef enum {
+    NVFP4_RULE_MAXERR = 0,     /* smaller maximum absolute error                           */
+    NVFP4_RULE_MAE = 1,        /* smaller mean absolute error                              */
+    NVFP4_RULE_MSE = 2         /* smaller mean squared error                               */
+} nvfp4_rule;
+
+/* Per-group absolute maximum (the input of the global tensor scale, [FOS] Implementation
+ * details). amax[g] = max |x| over group g, exactly (a BF16 value as binary32).
+ *   x     [groups, rows, cols] BF16 bits, 32-byte aligned          (in)
+ *   amax  [groups] float                                            (out)
+ * Enqueues a zero-fill of amax followed by one reduction kernel. An empty tensor writes
+ * amax = 0 for every group. */
+NVFP4_API nvfp4_status nvfp4_amax(const uint16_t* x, int64_t groups, int64_t rows, int64_t cols,
+                        float* amax, cudaStream_t stream);
+
+/* Quantize to NVFP4 ([FOS] Problem definition, Core mechanism, Adaptive block scaling
+ * algorithm, Implementation details). One kernel, one pass over x.
+ *   x       [groups, rows, cols] BF16 bits, 32-byte aligned                        (in)
+ *   amax    [groups] float, e.g. from nvfp4_amax, or a calibrated static value:
+ *           a value below the true maximum saturates the largest blocks              (in)
+ *   mode    NVFP4_SCALE6 or NVFP4_FOUR_OVER_SIX
+ *   rule    error rule; ignored (not validated) in scale-6 mode
+ *   codes   [groups*rows*cols/2] bytes: element 2j in the low nibble of byte j,
+ *           element 2j+1 in the high nibble, 8-byte aligned                          (out)
+ *   scales  [groups*rows*cols/16] E4M3 bytes, one per block, row-major              (out)
+ *   tscale  [groups] float alpha_g                                                  (out)
+ *   choice  NULL, or [ceil(groups*rows*cols/16 / 8)] bytes, 4-byte aligned: bit b%8 of
+ *           byte b/8 set iff block b (flat index) kept target 4; all zero in scale-6 (out)
+ * An empty tensor writes tscale[g] = alpha of amax[g] for every group (nothing else). */
+NVFP4_API nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t groups, int64_t rows, int64_t cols,
+                            const float* amax, nvfp4_mode mode, nvfp4_rule rule,
+                            uint8_t* codes, uint8_t* scales, float* tscale, uint8_t* choice,
+                            cudaStream_t stream);
+
+/* Dequantize NVFP4 to BF16: y_i = bf16_rne(v(c_i) * (f32(s_b) * alpha_g)), the values the
+ * stored tensor represents ([FOS] Problem definition; block and tensor scales of
+ * Implementation details).
+ *   codes, scales, tscale as written by nvfp4_quantize                              (in)
+ *   y       [groups, rows, cols] BF16 bits, 32-byte aligned                          (out)
+ * An empty tensor does nothing. */
+NVFP4_API nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tscale,
+                              int64_t groups, int64_t rows, int64_t cols, uint16_t* y,
+                              cudaStream_t stream);
+
+/* Fake quantization (quantize then dequantize in one pass): the simulated-quantization
+ * forward of a QAD student ([N35] two-stage QAD section). Bit-identical to
+ * nvfp4_quantize followed by nvfp4_dequantize, without materialising the codes.
+ *   x, amax, mode, rule as for nvfp4_quantize                                         (in)
+ *   y       [groups, rows, cols] BF16 bits, 32-byte aligned                           (out)
+ *   choice  NULL or the choice bitmap as for nvfp4_quantize                           (out)
+ * An empty tensor does nothing. */
+NVFP4_API nvfp4_status nvfp4_fakequant(const uint16_t* x, int64_t groups, int64_t rows, int64_t cols,
+                             const float* amax, nvfp4_mode mode, nvfp4_rule rule,
+                             uint16_t* y, uint8_t* choice, cudaStream_t stream);
+
+/* Static description of a status code (never NULL). */
+NVFP4_API const char* nvfp4_status_string(nvfp4_status status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+NVFP4_API int nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_H */

@@ -1,0 +1,207 @@
+"""Python binding of libnvfp4.so (include/nvfp4.h): BF16 -> NVFP4 quantization on B200.
+
+The functions named ``nvfp4_*`` mirror the C ABI one to one and only marshal arguments:
+torch CUDA tensors in, device pointers and the current CUDA stream out. Every step of the
+computation runs in the library's sm_100a kernels; there is no CPU path. If the shared
+library is missing, ``load()`` raises.
+
+The convenience wrappers ``quantize``, ``fakequant`` and ``dequantize`` allocate outputs
+with torch and call the same entry points.
+
+Sources: "Four Over Six: More Accurate NVFP4 Quantization with Adaptive Block Scaling"
+(gist.science explainer), technical summary (Problem definition; Method; Implementation
+details); "Quantization-Aware Distillation for NVFP4 Inference Accuracy Recovery" §3.3
+(blocks of 16).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import NamedTuple
+
+__all__ = [
+    "load", "library_path", "Nvfp4Error",
+    "SCALE6", "FOUR_OVER_SIX", "RULE_MAXERR", "RULE_MAE", "RULE_MSE",
+    "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fakequant",
+    "nvfp4_status_string", "nvfp4_version",
+    "Quantized", "amax", "quantize", "fakequant", "dequantize",
+]
+
+SCALE6, FOUR_OVER_SIX = 0, 1
+RULE_MAXERR, RULE_MAE, RULE_MSE = 0, 1, 2
+_MODES = {"scale6": SCALE6, "four_over_six": FOUR_OVER_SIX, "4/6": FOUR_OVER_SIX}
+_RULES = {"maxerr": RULE_MAXERR, "max": RULE_MAXERR, "mae": RULE_MAE, "mse": RULE_MSE}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "lib", "libnvfp4.so")
+_lib = None
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, status: int, func: str):
+        self.status = status
+        super().__init__(f"{func}: {nvfp4_status_string(status)} (status {status})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load libnvfp4.so (built by ``python -m nvfp4_block_scaled_13_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"libnvfp4.so not built: {_LIB_PATH} is missing "
+                              "(run python -m nvfp4_block_scaled_13_b200.build)")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        L.nvfp4_amax.argtypes = [vp, i64, i64, i64, vp, vp]
+        L.nvfp4_quantize.argtypes = [vp, i64, i64, i64, vp, i32, i32, vp, vp, vp, vp, vp]
+        L.nvfp4_dequantize.argtypes = [vp, vp, vp, i64, i64, i64, vp, vp]
+        L.nvfp4_fakequant.argtypes = [vp, i64, i64, i64, vp, i32, i32, vp, vp, vp]
+        for f in (L.nvfp4_amax, L.nvfp4_quantize, L.nvfp4_dequantize, L.nvfp4_fakequant):
+            f.restype = i32
+        L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
+        L.nvfp4_version.argtypes, L.nvfp4_version.restype = [], i32
+        _lib = L
+    return _lib
+
+
+# ---- marshalling helpers -------------------------------------------------------------------
+
+def _ptr(t):
+    """Device pointer of a CUDA tensor (None -> NULL). Raw integers pass through."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("nvfp4: tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("nvfp4: tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, func: str):
+    if status != 0:
+        raise Nvfp4Error(status, func)
+
+
+def _mode(m):
+    return _MODES[m] if isinstance(m, str) else int(m)
+
+
+def _rule(r):
+    return _RULES[r] if isinstance(r, str) else int(r)
+
+
+# ---- the C ABI, one to one -------------------------------------------------------------------
+
+def nvfp4_amax(x, groups, rows, cols, amax, stream=None):
+    _check(load().nvfp4_amax(_ptr(x), groups, rows, cols, _ptr(amax), _stream(stream)), "nvfp4_amax")
+
+
+def nvfp4_quantize(x, groups, rows, cols, amax, mode, rule, codes, scales, tscale, choice=None, stream=None):
+    _check(load().nvfp4_quantize(_ptr(x), groups, rows, cols, _ptr(amax), _mode(mode), _rule(rule),
+                                 _ptr(codes), _ptr(scales), _ptr(tscale), _ptr(choice), _stream(stream)),
+           "nvfp4_quantize")
+
+
+def nvfp4_dequantize(codes, scales, tscale, groups, rows, cols, y, stream=None):
+    _check(load().nvfp4_dequantize(_ptr(codes), _ptr(scales), _ptr(tscale), groups, rows, cols, _ptr(y),
+                                   _stream(stream)), "nvfp4_dequantize")
+
+
+def nvfp4_fakequant(x, groups, rows, cols, amax, mode, rule, y, choice=None, stream=None):
+    _check(load().nvfp4_fakequant(_ptr(x), groups, rows, cols, _ptr(amax), _mode(mode), _rule(rule),
+                                  _ptr(y), _ptr(choice), _stream(stream)), "nvfp4_fakequant")
+
+
+def nvfp4_status_string(status: int) -> str:
+    return load().nvfp4_status_string(int(status)).decode()
+
+
+def nvfp4_version() -> int:
+    return load().nvfp4_version()
+
+
+# ---- convenience wrappers (torch allocates, the library computes) -----------------------------
+
+class Quantized(NamedTuple):
+    codes: "object"      # uint8 [groups*rows*cols/2]
+    scales: "object"     # uint8 [groups*rows*cols/16] (E4M3 bits)
+    tscale: "object"     # float32 [groups]
+    choice: "object"     # uint8 [ceil(blocks/8)] or None
+    shape: tuple         # (groups, rows, cols)
+
+
+def _shape3(x, groups):
+    if x.dtype.itemsize != 2:
+        raise ValueError("nvfp4: x must be BF16 (or its uint16/int16 bits)")
+    cols = x.shape[-1] if x.dim() > 0 else 0
+    n = x.numel()
+    if groups < 1 or (cols and n % (groups * cols)):
+        raise ValueError("nvfp4: numel must be a multiple of groups * cols")
+    rows = n // (groups * cols) if cols else 0
+    return groups, rows, cols
+
+
+def amax(x, groups: int = 1, stream=None):
+    import torch
+
+    g, r, c = _shape3(x, groups)
+    out = torch.empty(g, dtype=torch.float32, device=x.device)
+    nvfp4_amax(x, g, r, c, out, stream)
+    return out
+
+
+def quantize(x, mode="four_over_six", rule="mse", groups: int = 1, amax_values=None, with_choice=True,
+             stream=None) -> Quantized:
+    import torch
+
+    g, r, c = _shape3(x, groups)
+    if amax_values is None:
+        amax_values = amax(x, groups, stream)
+    n = g * r * c
+    nb = n // 16
+    dev = x.device
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(nb, dtype=torch.uint8, device=dev)
+    tscale = torch.empty(g, dtype=torch.float32, device=dev)
+    choice = torch.empty(max(1, (nb + 7) // 8), dtype=torch.uint8, device=dev) if with_choice else None
+    nvfp4_quantize(x, g, r, c, amax_values, mode, rule, codes, scales, tscale, choice, stream)
+    return Quantized(codes, scales, tscale, choice, (g, r, c))
+
+
+def dequantize(q: Quantized, out=None, stream=None):
+    import torch
+
+    g, r, c = q.shape
+    if out is None:
+        out = torch.empty((g * r, c) if c else (0,), dtype=torch.bfloat16, device=q.codes.device)
+    nvfp4_dequantize(q.codes, q.scales, q.tscale, g, r, c, out, stream)
+    return out
+
+
+def fakequant(x, mode="four_over_six", rule="mse", groups: int = 1, amax_values=None, out=None, choice=None,
+              stream=None):
+    import torch
+
+    g, r, c = _shape3(x, groups)
+    if amax_values is None:
+        amax_values = amax(x, groups, stream)
+    if out is None:
+        out = torch.empty_like(x, dtype=torch.bfloat16)
+    nvfp4_fakequant(x, g, r, c, amax_values, mode, rule, out, choice, stream)
+    return out

@@ -1,0 +1,254 @@
+// nvfp4_api.cu — the C ABI declared in include/nvfp4.h: argument validation, launch
+// configuration and kernel dispatch. No allocation, no host synchronization, no state
+// beyond a per-device cache of launch limits.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+
+#include "../../include/nvfp4.h"
+#include "kernels.cuh"
+
+namespace {
+
+using nvfp4::GroupDiv;
+using nvfp4::kThreads;
+
+constexpr int kMaxDevices = 64;
+
+// Launch limits of one device: SM count and resident CTAs per SM for each kernel family.
+struct DeviceInfo {
+    std::atomic<int> sms{0};
+};
+DeviceInfo g_dev[kMaxDevices];
+
+int sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev >= kMaxDevices) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        return n > 0 ? n : 148;
+    }
+    int n = g_dev[dev].sms.load(std::memory_order_relaxed);
+    if (n == 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        g_dev[dev].sms.store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
+// Resident CTAs per SM for a kernel, cached per kernel instantiation and device.
+template <typename Kernel>
+int ctas_per_sm(Kernel kernel) {
+    static std::atomic<int> cache[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int v = (dev >= 0 && dev < kMaxDevices) ? cache[dev].load(std::memory_order_relaxed) : 0;
+    if (v == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kernel, kThreads, 0) != cudaSuccess || v <= 0) v = 1;
+        if (dev >= 0 && dev < kMaxDevices) cache[dev].store(v, std::memory_order_relaxed);
+    }
+    return v;
+}
+
+// Persistent grid: enough CTAs to fill every SM at full occupancy, never more than the work.
+template <typename Kernel>
+unsigned grid_for(Kernel kernel, int64_t work_items) {
+    const int64_t full = static_cast<int64_t>(sm_count()) * ctas_per_sm(kernel);
+    const int64_t need = (work_items + kThreads - 1) / kThreads;
+    const int64_t g = need < full ? need : full;
+    return static_cast<unsigned>(g < 1 ? 1 : g);
+}
+
+GroupDiv make_gdiv(int64_t groups, int64_t bpg, int64_t nblocks) {
+    GroupDiv d{};
+    d.bpg = bpg;
+    if (groups == 1) {
+        d.mode = 0;
+    } else if (bpg == 1) {
+        d.mode = 1;
+    } else if (nblocks < (int64_t(1) << 31) && bpg < (int64_t(1) << 31)) {
+        // q = floor(b * m / 2^(31 + l)) with m = ceil(2^(31 + l) / bpg), l = ceil(log2 bpg):
+        // exact for every b < 2^31, and m < 2^32 because bpg > 2^(l - 1).
+        uint32_t l = 0;
+        while ((int64_t(1) << l) < bpg) ++l;
+        const unsigned __int128 num = (unsigned __int128)1 << (31 + l);
+        d.mul = static_cast<uint32_t>((num + bpg - 1) / bpg);
+        d.shift = l - 1;
+        d.mode = 2;
+    } else {
+        d.mode = 3;
+    }
+    return d;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Shared shape check. Returns NVFP4_OK and the element count, or an error.
+nvfp4_status check_shape(int64_t groups, int64_t rows, int64_t cols, int64_t* numel) {
+    if (groups < 1 || rows < 0 || cols < 0 || cols % 16 != 0) return NVFP4_ERR_SHAPE;
+    const int64_t lim = int64_t(1) << 62;
+    if (rows > 0 && cols > lim / rows) return NVFP4_ERR_SHAPE;
+    const int64_t per = rows * cols;
+    if (per > 0 && groups > lim / per) return NVFP4_ERR_SHAPE;
+    *numel = groups * per;
+    return NVFP4_OK;
+}
+
+nvfp4_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+template <bool FOUR, int RULE, bool FQ>
+nvfp4_status launch_quant(const nvfp4::QuantParams& p, cudaStream_t stream) {
+    auto kernel = nvfp4::quantize_kernel<FOUR, RULE, FQ>;
+    const unsigned grid = grid_for(kernel, p.nblocks);
+    kernel<<<grid, kThreads, 0, stream>>>(p);
+    return launch_status();
+}
+
+template <bool FQ>
+nvfp4_status dispatch_quant(nvfp4_mode mode, nvfp4_rule rule, const nvfp4::QuantParams& p, cudaStream_t s) {
+    if (mode == NVFP4_SCALE6) return launch_quant<false, nvfp4::kMse, FQ>(p, s);
+    switch (rule) {
+        case NVFP4_RULE_MAXERR: return launch_quant<true, nvfp4::kMaxErr, FQ>(p, s);
+        case NVFP4_RULE_MAE: return launch_quant<true, nvfp4::kMae, FQ>(p, s);
+        default: return launch_quant<true, nvfp4::kMse, FQ>(p, s);
+    }
+}
+
+nvfp4_status check_mode_rule(nvfp4_mode mode, nvfp4_rule rule) {
+    if (mode != NVFP4_SCALE6 && mode != NVFP4_FOUR_OVER_SIX) return NVFP4_ERR_MODE;
+    if (mode == NVFP4_FOUR_OVER_SIX && rule != NVFP4_RULE_MAXERR && rule != NVFP4_RULE_MAE && rule != NVFP4_RULE_MSE)
+        return NVFP4_ERR_RULE;
+    return NVFP4_OK;
+}
+
+// alpha_g = amax_g / (6 M) for empty tensors (no blocks to quantize).
+__global__ void tensor_scale_only_kernel(const float* amax, float* tscale, int64_t groups, float six_m) {
+    for (int64_t g = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; g < groups; g += int64_t(gridDim.x) * blockDim.x)
+        tscale[g] = __fdiv_rn(amax[g], six_m);
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_amax(const uint16_t* x, int64_t groups, int64_t rows, int64_t cols, float* amax,
+                        cudaStream_t stream) {
+    if (amax == nullptr) return NVFP4_ERR_NULL;
+    int64_t n = 0;
+    nvfp4_status st = check_shape(groups, rows, cols, &n);
+    if (st != NVFP4_OK) return st;
+    if (n > 0 && x == nullptr) return NVFP4_ERR_NULL;
+    if (!aligned(amax, 4) || (n > 0 && !aligned(x, 32))) return NVFP4_ERR_ALIGN;
+    if (cudaMemsetAsync(amax, 0, static_cast<size_t>(groups) * sizeof(float), stream) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    if (n == 0) return launch_status();
+    const int64_t chunks = rows * cols / 16;
+    const int64_t full = static_cast<int64_t>(sm_count()) * ctas_per_sm(nvfp4::amax_kernel);
+    int64_t per_group = full / groups;
+    if (per_group < 1) per_group = 1;
+    const int64_t need = (chunks + kThreads - 1) / kThreads;
+    if (per_group > need) per_group = need;
+    const int64_t gy = groups < 65535 ? groups : 65535;
+    dim3 grid(static_cast<unsigned>(per_group), static_cast<unsigned>(gy));
+    nvfp4::amax_kernel<<<grid, kThreads, 0, stream>>>(x, groups, chunks, amax);
+    return launch_status();
+}
+
+nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t groups, int64_t rows, int64_t cols, const float* amax,
+                            nvfp4_mode mode, nvfp4_rule rule, uint8_t* codes, uint8_t* scales, float* tscale,
+                            uint8_t* choice, cudaStream_t stream) {
+    if (amax == nullptr || tscale == nullptr) return NVFP4_ERR_NULL;
+    int64_t n = 0;
+    nvfp4_status st = check_shape(groups, rows, cols, &n);
+    if (st != NVFP4_OK) return st;
+    if (n > 0 && (x == nullptr || codes == nullptr || scales == nullptr)) return NVFP4_ERR_NULL;
+    st = check_mode_rule(mode, rule);
+    if (st != NVFP4_OK) return st;
+    if (!aligned(amax, 4) || !aligned(tscale, 4) || (choice && !aligned(choice, 4))) return NVFP4_ERR_ALIGN;
+    if (n > 0 && (!aligned(x, 32) || !aligned(codes, 8))) return NVFP4_ERR_ALIGN;
+    const float six_m = mode == NVFP4_FOUR_OVER_SIX ? 1536.0f : 2688.0f;
+    if (n == 0) {
+        const unsigned grid = static_cast<unsigned>((groups + kThreads - 1) / kThreads < 1024 ? (groups + kThreads - 1) / kThreads : 1024);
+        tensor_scale_only_kernel<<<grid, kThreads, 0, stream>>>(amax, tscale, groups, six_m);
+        return launch_status();
+    }
+    nvfp4::QuantParams p{};
+    p.x = x;
+    p.amax = amax;
+    p.codes = codes;
+    p.scales = scales;
+    p.tscale = tscale;
+    p.choice = choice;
+    p.y = nullptr;
+    p.nblocks = n / 16;
+    p.choice_bytes = (p.nblocks + 7) / 8;
+    p.gdiv = make_gdiv(groups, rows * cols / 16, p.nblocks);
+    if (mode == NVFP4_SCALE6 && choice != nullptr) {
+        // the kernel's ballot writes zero words; nothing else is needed
+    }
+    return dispatch_quant<false>(mode, rule, p, stream);
+}
+
+nvfp4_status nvfp4_fakequant(const uint16_t* x, int64_t groups, int64_t rows, int64_t cols, const float* amax,
+                             nvfp4_mode mode, nvfp4_rule rule, uint16_t* y, uint8_t* choice, cudaStream_t stream) {
+    if (amax == nullptr) return NVFP4_ERR_NULL;
+    int64_t n = 0;
+    nvfp4_status st = check_shape(groups, rows, cols, &n);
+    if (st != NVFP4_OK) return st;
+    if (n > 0 && (x == nullptr || y == nullptr)) return NVFP4_ERR_NULL;
+    st = check_mode_rule(mode, rule);
+    if (st != NVFP4_OK) return st;
+    if (!aligned(amax, 4) || (choice && !aligned(choice, 4))) return NVFP4_ERR_ALIGN;
+    if (n > 0 && (!aligned(x, 32) || !aligned(y, 32))) return NVFP4_ERR_ALIGN;
+    if (n == 0) return NVFP4_OK;
+    nvfp4::QuantParams p{};
+    p.x = x;
+    p.amax = amax;
+    p.choice = choice;
+    p.y = y;
+    p.nblocks = n / 16;
+    p.choice_bytes = (p.nblocks + 7) / 8;
+    p.gdiv = make_gdiv(groups, rows * cols / 16, p.nblocks);
+    return dispatch_quant<true>(mode, rule, p, stream);
+}
+
+nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tscale, int64_t groups,
+                              int64_t rows, int64_t cols, uint16_t* y, cudaStream_t stream) {
+    int64_t n = 0;
+    nvfp4_status st = check_shape(groups, rows, cols, &n);
+    if (st != NVFP4_OK) return st;
+    if (n == 0) return NVFP4_OK;
+    if (codes == nullptr || scales == nullptr || tscale == nullptr || y == nullptr) return NVFP4_ERR_NULL;
+    if (!aligned(codes, 8) || !aligned(tscale, 4) || !aligned(y, 32)) return NVFP4_ERR_ALIGN;
+    nvfp4::DequantParams p{};
+    p.codes = codes;
+    p.scales = scales;
+    p.tscale = tscale;
+    p.y = y;
+    p.nblocks = n / 16;
+    p.gdiv = make_gdiv(groups, rows * cols / 16, p.nblocks);
+    const unsigned grid = grid_for(nvfp4::dequantize_kernel, p.nblocks);
+    nvfp4::dequantize_kernel<<<grid, kThreads, 0, stream>>>(p);
+    return launch_status();
+}
+
+const char* nvfp4_status_string(nvfp4_status status) {
+    switch (status) {
+        case NVFP4_OK: return "ok";
+        case NVFP4_ERR_NULL: return "a required pointer is NULL";
+        case NVFP4_ERR_SHAPE: return "invalid shape (groups >= 1, rows/cols >= 0, cols % 16 == 0, size limit)";
+        case NVFP4_ERR_ALIGN: return "misaligned pointer (BF16 tensors 32 B, codes 8 B, floats and choice 4 B)";
+        case NVFP4_ERR_MODE: return "unknown nvfp4_mode";
+        case NVFP4_ERR_RULE: return "unknown nvfp4_rule";
+        case NVFP4_ERR_CUDA: return "CUDA runtime error while enqueuing work";
+        default: return "unknown nvfp4_status";
+    }
+}
+
+int nvfp4_version(void) { return 100; }
+
+}  // extern "C"

@@ -49,6 +49,8 @@ def lib():
         L.nvo_e4m3_to_f32.argtypes, L.nvo_e4m3_to_f32.restype = [u8], f32
         L.nvo_f32_to_e2m1_satfinite.argtypes, L.nvo_f32_to_e2m1_satfinite.restype = [f32], u8
         L.nvo_e2m1_to_f32.argtypes, L.nvo_e2m1_to_f32.restype = [u8], f32
+        for name in ("nvo_f32_to_e2m1_array", "nvo_f32_to_e4m3_array", "nvo_f32_to_bf16_array"):
+            getattr(L, name).argtypes, getattr(L, name).restype = [vp, vp, i64], None
         L.nvo_block_candidate.argtypes = [vp, f32, f32, i32, ctypes.POINTER(Candidate)]
         L.nvo_block_candidate.restype = None
         L.nvo_amax.argtypes, L.nvo_amax.restype = [vp, i64, i64, i64, vp], None
@@ -100,6 +102,27 @@ def f32_to_bf16(f) -> np.ndarray:
     f = np.asarray(f, dtype=np.float32).ravel()
     L = lib()
     return np.array([L.nvo_f32_to_bf16_rne(float(v)) for v in f], dtype=np.uint16)
+
+
+def f32_to_e2m1_array(a: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    out = np.empty(a.size, np.uint8)
+    lib().nvo_f32_to_e2m1_array(_ptr(a), _ptr(out), a.size)
+    return out
+
+
+def f32_to_e4m3_array(a: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    out = np.empty(a.size, np.uint8)
+    lib().nvo_f32_to_e4m3_array(_ptr(a), _ptr(out), a.size)
+    return out
+
+
+def f32_to_bf16_array(a: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    out = np.empty(a.size, np.uint16)
+    lib().nvo_f32_to_bf16_array(_ptr(a), _ptr(out), a.size)
+    return out
 
 
 def block_candidate(x16, alpha: float, K: float, rule: int) -> Candidate:

@@ -125,6 +125,18 @@ float nvo_e2m1_to_f32(uint8_t c) {
     return (float)((c & 0x8u) ? -v : v);
 }
 
+void nvo_f32_to_e2m1_array(const float* in, uint8_t* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = nvo_f32_to_e2m1_satfinite(in[i]);
+}
+
+void nvo_f32_to_e4m3_array(const float* in, uint8_t* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = nvo_f32_to_e4m3_satfinite(in[i]);
+}
+
+void nvo_f32_to_bf16_array(const float* in, uint16_t* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = nvo_f32_to_bf16_rne(in[i]);
+}
+
 /* ---- one block, one candidate --------------------------------------------------------- */
 
 void nvo_block_candidate(const float x[16], float alpha, float K, int rule, nvo_candidate* c) {

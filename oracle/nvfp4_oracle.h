@@ -59,6 +59,11 @@ uint8_t nvo_f32_to_e2m1_satfinite(float y);
 /* 4-bit E2M1 code -> binary32 (exact). */
 float nvo_e2m1_to_f32(uint8_t c);
 
+/* Element-wise array versions of the conversions above (for exhaustive comparisons). */
+void nvo_f32_to_e2m1_array(const float* in, uint8_t* out, int64_t n);
+void nvo_f32_to_e4m3_array(const float* in, uint8_t* out, int64_t n);
+void nvo_f32_to_bf16_array(const float* in, uint16_t* out, int64_t n);
+
 /* ---- one 16-element block, one candidate ---------------------------------------------- */
 
 typedef struct {

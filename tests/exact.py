@@ -73,3 +73,25 @@ def nearest_ties_even(v: F, table):
     mids = [(table[k] + table[k + 1]) / 2 for k in range(len(table) - 1)]
     margin = min(abs(v - mp) for mp in mids)
     return i, margin
+
+
+def round_f32(v: F) -> F:
+    """Round an exact rational to the nearest binary32 (ties to even); overflow -> None."""
+    if v == 0:
+        return F(0)
+    sign = -1 if v < 0 else 1
+    a = abs(v)
+    # exponent e with 2^e <= a < 2^(e+1)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if F(2) ** e > a:
+        e -= 1
+    q = F(2) ** (max(e, -126) - 23)       # quantum of that binade (subnormals below 2^-126)
+    n = a / q
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    if rem > F(1, 2) or (rem == F(1, 2) and fl % 2 == 1):
+        fl += 1
+    r = fl * q
+    if r > FLT_MAX:
+        return None
+    return sign * r
