@@ -28,7 +28,8 @@
  *       s    = E4M3(t), round to nearest even, saturating at 448
  *       d    = f32(s) * alpha;  r = (d > 0) ? min(1 / d, FLT_MAX) : 0
  *       c_i  = E2M1(x_i * r), round to nearest even, saturating at 6, sign kept
- *       q_i  = v(c_i) * d;  e_i = x_i - q_i   (error against the original values)
+ *       q_i  = v(c_i) * d;  e_i = x_i - v(c_i) * d, the exact difference rounded once
+ *              (a fused multiply-add): the error against the original values
  *       err  = MAXERR: max |e_i|;  MAE: S(|e_i|);  MSE: S(e_i^2) with fused multiply-add,
  *              where S sums even-indexed and odd-indexed terms in two running sums (each in
  *              increasing index order, starting from +0) and then adds the two

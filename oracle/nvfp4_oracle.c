@@ -168,8 +168,11 @@ void nvo_block_candidate(const float x[16], float alpha, float K, int rule, nvo_
     for (int i = 0; i < 16; ++i) {
         float y = x[i] * c->r;
         c->code[i] = nvo_f32_to_e2m1_satfinite(y);
-        c->q[i] = nvo_e2m1_to_f32(c->code[i]) * c->d;
-        c->e[i] = x[i] - c->q[i];
+        float v = nvo_e2m1_to_f32(c->code[i]);
+        c->q[i] = v * c->d;
+        /* Reading: the error is the exact difference between the original value and the
+         * dequantized value v * d, rounded once (a fused multiply-add). */
+        c->e[i] = fmaf(-v, c->d, x[i]);
         float ae = fabsf(c->e[i]);
         /* Rules (Adaptive block scaling algorithm: selection rule). Reading: sums are not
          * divided by 16 (an exact scaling that cannot change the choice) and are accumulated

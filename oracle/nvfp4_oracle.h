@@ -18,7 +18,8 @@
  *          two-stage QAD process (the student's forward runs through simulated quantization).
  *
  * Arithmetic: IEEE-754 binary32, round-to-nearest-even for every operation, no fused
- * multiply-add except the explicit fmaf of the MSE rule, subnormals kept (no FTZ/DAZ).
+ * multiply-add except the explicit fmaf calls (the error x - v*d and the MSE sum),
+ * subnormals kept (no FTZ/DAZ).
  * Built with -O2 -fno-fast-math -ffp-contract=off. The narrow formats (E2M1, E4M3, BF16)
  * are converted by exact lattice arithmetic in binary64, written from their definitions.
  *
@@ -74,7 +75,7 @@ typedef struct {
     float    r;         /* encode factor: 0 if d == 0, else min(1/d, FLT_MAX)            */
     uint8_t  code[16];  /* E2M1 codes of x_i * r                                        */
     float    q[16];     /* dequantized values v(code_i) * d (rounded once)              */
-    float    e[16];     /* errors x_i - q_i (rounded once)                              */
+    float    e[16];     /* errors x_i - v(code_i) * d (exact difference, rounded once)  */
     float    err;       /* the rule's error: max|e|, sum|e| or sum e^2 (see below)       */
 } nvo_candidate;
 

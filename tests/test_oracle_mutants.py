@@ -31,7 +31,8 @@ MUTANTS = {
     "nibbles_swapped": ("(uint8_t)(chosen->code[2 * j] | (chosen->code[2 * j + 1] << 4))",
                         "(uint8_t)(chosen->code[2 * j + 1] | (chosen->code[2 * j] << 4))"),
     "decode_scale_transposed": ("c->d = nvo_e4m3_to_f32(c->s) * alpha;", "c->d = nvo_e4m3_to_f32(c->s) / alpha;"),
-    "error_against_scaled_values": ("c->e[i] = x[i] - c->q[i];", "c->e[i] = y - nvo_e2m1_to_f32(c->code[i]);"),
+    "error_against_scaled_values": ("c->e[i] = fmaf(-v, c->d, x[i]);", "c->e[i] = y - v;"),
+    "error_drops_scale": ("c->e[i] = fmaf(-v, c->d, x[i]);", "c->e[i] = x[i] - v;"),
     "zero_sign_dropped": ("uint8_t sign = signbit(y) ? 0x8u : 0x0u;", "uint8_t sign = (y < 0) ? 0x8u : 0x0u;"),
 }
 
