@@ -113,27 +113,24 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
 
 // ---- quantize / fake-quant -----------------------------------------------------------------
 
-// One candidate (target maximum K) of one block: codes, dequantized values and the rule's
-// error. The two running sums of MAE/MSE are the two lanes of a packed pair (even and odd
-// element indices), added at the end.
+// One candidate (target maximum K) of one block: its codes, their exact values as f16x2
+// words, and the rule's error. e_i = x_i - v_i * d is one fused multiply-add (the exact
+// difference, rounded once). The two running sums of MAE/MSE are the two lanes of a packed
+// pair (even and odd element indices), added at the end.
 template <int RULE>
 __device__ __forceinline__ float candidate(const float2 (&x)[8], float r, float d, uint32_t& c_lo,
-                                           uint32_t& c_hi, float2 (&q)[8]) {
-    const float2 rr = make_float2(r, r), dd = make_float2(d, d);
+                                           uint32_t& c_hi, uint32_t (&h)[8]) {
+    const float2 rr = make_float2(r, r), nd = make_float2(-d, -d);
     float2 y[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) y[j] = mul2(x[j], rr);
-    c_lo = e2m1x8(y[0], y[1], y[2], y[3]);
-    c_hi = e2m1x8(y[4], y[5], y[6], y[7]);
-    uint32_t h[8];
-    e2m1x8_to_f16x2(c_lo, h[0], h[1], h[2], h[3]);
-    e2m1x8_to_f16x2(c_hi, h[4], h[5], h[6], h[7]);
+    c_lo = e2m1x8_and_decode(y[0], y[1], y[2], y[3], h[0], h[1], h[2], h[3]);
+    c_hi = e2m1x8_and_decode(y[4], y[5], y[6], y[7], h[4], h[5], h[6], h[7]);
     float2 acc = make_float2(0.0f, 0.0f);
     float emax = 0.0f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        q[j] = mul2(f16x2_to_float2(h[j]), dd);
-        const float2 e = sub2(x[j], q[j]);
+        const float2 e = fma2(f16x2_to_float2(h[j]), nd, x[j]);
         if (RULE == kMse) {
             acc = fma2(e, e, acc);
         } else if (RULE == kMae) {
@@ -196,31 +193,29 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p)
             const uint32_t s2 = e4m3x2(t6, t4);
             const float2 sf = e4m3x2_to_float2(s2);
             const float d6 = __fmul_rn(sf.x, alpha);
-            uint32_t c6lo, c6hi;
-            float2 q6[8];
-            const float err6 = candidate<RULE>(x, recip_clamped(d6), d6, c6lo, c6hi, q6);
+            uint32_t c6lo, c6hi, h[8];
+            const float err6 = candidate<RULE>(x, recip_clamped(d6), d6, c6lo, c6hi, h);
             uint32_t clo = c6lo, chi = c6hi, s = s2 & 0xFFu;
-            float2 qsel[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) qsel[j] = q6[j];
+            float dsel = d6;
             if (FOUR) {
                 const float d4 = __fmul_rn(sf.y, alpha);
-                uint32_t c4lo, c4hi;
-                float2 q4[8];
-                const float err4 = candidate<RULE>(x, recip_clamped(d4), d4, c4lo, c4hi, q4);
+                uint32_t c4lo, c4hi, h4[8];
+                const float err4 = candidate<RULE>(x, recip_clamped(d4), d4, c4lo, c4hi, h4);
                 four = err4 < err6;   // ties keep target 6
                 if (four) {
                     clo = c4lo;
                     chi = c4hi;
                     s = s2 >> 8;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) qsel[j] = q4[j];
+                    dsel = d4;
                 }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) h[j] = four ? h4[j] : h[j];
             }
-            if (FQ) {
+            if (FQ) {   // q = RN(v * d) of the kept candidate, rounded to BF16
+                const float2 dd = make_float2(dsel, dsel);
                 uint32_t out[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) out[j] = bf16x2(qsel[j]);
+                for (int j = 0; j < 8; ++j) out[j] = bf16x2(mul2(f16x2_to_float2(h[j]), dd));
                 st32(p.y + b * 16, out);
             } else {
                 st8(p.codes + b * 8, clo, chi);

@@ -88,24 +88,33 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
 
 // ---- format conversions ------------------------------------------------------------------
 
-// Eight binary32 values (four pairs p[j] = (element 2j, element 2j+1)) -> eight E2M1 codes,
-// packed so that element k sits in bits [4k, 4k+4): the low nibble of each byte holds the
-// even element. cvt ... d, a, b puts a in the high nibble and b in the low nibble.
-__device__ __forceinline__ uint32_t e2m1x8(float2 p0, float2 p1, float2 p2, float2 p3) {
+// Eight binary32 values (four pairs p[j] = (element 2j, element 2j+1)) -> eight E2M1 codes
+// packed so that element k sits in bits [4k, 4k+4) (the low nibble of each byte holds the
+// even element; cvt ... d, a, b puts a in the high nibble and b in the low nibble), and the
+// codes' exact values as four f16x2 words (word j: element 2j low, 2j+1 high).
+// The decode reads the .b8 results of the conversions inside the same asm block: decoding
+// bytes that were first packed into a 32-bit word and unpacked again gave zeros for bytes 2
+// and 3 on sm_100a, so this pattern is avoided.
+__device__ __forceinline__ uint32_t e2m1x8_and_decode(float2 p0, float2 p1, float2 p2, float2 p3, uint32_t& h0,
+                                                      uint32_t& h1, uint32_t& h2, uint32_t& h3) {
     uint32_t r;
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %8, %7;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %10, %9;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %12, %11;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %4, b3;\n\t"
         "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-        : "=r"(r)
+        : "=r"(r), "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
         : "f"(p0.x), "f"(p0.y), "f"(p1.x), "f"(p1.y), "f"(p2.x), "f"(p2.y), "f"(p3.x), "f"(p3.y));
     return r;
 }
 
-// Eight packed E2M1 codes -> four f16x2 words (exact); word j holds elements 2j (low half)
-// and 2j+1 (high half).
+// Eight packed E2M1 codes loaded from memory -> four f16x2 words (exact); word j holds
+// elements 2j (low half) and 2j+1 (high half).
 __device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t& h0, uint32_t& h1, uint32_t& h2,
                                                 uint32_t& h3) {
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"

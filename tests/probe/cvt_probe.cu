@@ -64,7 +64,9 @@ __global__ void k_bf16(const float* in, uint16_t* out, int64_t n) {
     }
 }
 
-// op: 0 rcp_rn(a), 1 div_rn(a, b), 2 mul.rn.f32x2, 3 sub.rn.f32x2, 4 add.rn.f32x2, 5 fma.rn.f32x2(a, b, c)
+// op: 0 rcp_rn(a), 1 div_rn(a, b), 2 mul.rn.f32x2, 3 sub.rn.f32x2, 4 add.rn.f32x2, 5 fma.rn.f32x2(a, b, c),
+// 6 c - a*b written as mul.rn.f32x2 then sub.rn.f32x2 (two roundings expected),
+// 7 c - a*b written as fma.rn.f32x2(a, b, -0) then sub.rn.f32x2 (two roundings)
 __global__ void k_arith(int op, const float* a, const float* b, const float* c, float* out, int64_t n) {
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n / 2; i += int64_t(gridDim.x) * blockDim.x) {
         float a0 = a[2 * i], a1 = a[2 * i + 1], b0 = b[2 * i], b1 = b[2 * i + 1], c0 = c[2 * i], c1 = c[2 * i + 1];
@@ -84,10 +86,26 @@ __global__ void k_arith(int op, const float* a, const float* b, const float* c, 
                 asm("{ .reg .b64 x, y, z; mov.b64 x, {%2, %3}; mov.b64 y, {%4, %5}; add.rn.f32x2 z, x, y; mov.b64 {%0, %1}, z; }"
                     : "=f"(r0), "=f"(r1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
                 break;
-            default:
+            case 5:
                 asm("{ .reg .b64 x, y, w, z; mov.b64 x, {%2, %3}; mov.b64 y, {%4, %5}; mov.b64 w, {%6, %7}; fma.rn.f32x2 z, x, y, w; mov.b64 {%0, %1}, z; }"
                     : "=f"(r0), "=f"(r1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
                 break;
+            case 6: {
+                float p0, p1;
+                asm("{ .reg .b64 x, y, z; mov.b64 x, {%2, %3}; mov.b64 y, {%4, %5}; mul.rn.f32x2 z, x, y; mov.b64 {%0, %1}, z; }"
+                    : "=f"(p0), "=f"(p1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+                asm("{ .reg .b64 x, y, z; mov.b64 x, {%2, %3}; mov.b64 y, {%4, %5}; sub.rn.f32x2 z, x, y; mov.b64 {%0, %1}, z; }"
+                    : "=f"(r0), "=f"(r1) : "f"(c0), "f"(c1), "f"(p0), "f"(p1));
+                break;
+            }
+            default: {
+                float p0, p1;
+                asm("{ .reg .b64 x, y, w, z; mov.b64 x, {%2, %3}; mov.b64 y, {%4, %5}; mov.b64 w, {%6, %6}; fma.rn.f32x2 z, x, y, w; mov.b64 {%0, %1}, z; }"
+                    : "=f"(p0), "=f"(p1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(-0.0f));
+                asm("{ .reg .b64 x, y, z; mov.b64 x, {%2, %3}; mov.b64 y, {%4, %5}; sub.rn.f32x2 z, x, y; mov.b64 {%0, %1}, z; }"
+                    : "=f"(r0), "=f"(r1) : "f"(c0), "f"(c1), "f"(p0), "f"(p1));
+                break;
+            }
         }
         out[2 * i] = r0;
         out[2 * i + 1] = r1;

@@ -147,3 +147,20 @@ def test_packed_fma_is_single_rounding(probe):
     for i in range(a.size):
         want = X.round_f32(F(float(a[i])) * F(float(b[i])) + F(float(c[i])))
         assert want is not None and F(float(got[i])) == want, (a[i], b[i], c[i], got[i], float(want))
+
+
+def test_error_term_single_rounding(probe):
+    """x - v*d as the kernels compute it (one fused multiply-add, fma.rn.f32x2 with -d) is
+    the exact difference rounded once; the operands make that differ from rounding the
+    product first, so the data tells the two apart."""
+    rng = np.random.default_rng(31)
+    n = 200_000
+    v = rng.choice(np.array([0.5, 1, 1.5, 2, 3, 4, 6], np.float32), n).astype(np.float32)
+    d = (np.float32(1.0) + rng.random(n, dtype=np.float32)).astype(np.float32)
+    x = (v.astype(np.float64) * d * (1 + rng.standard_normal(n) * 1e-6)).astype(np.float32)
+    got = _arith(probe, 5, v, -d, x)
+    exact = x.astype(np.float64) - v.astype(np.float64) * d.astype(np.float64)   # exact: 24+3 bit product
+    want = exact.astype(np.float32)
+    two = x - v * d
+    assert int((want.view(np.uint32) != two.view(np.uint32)).sum()) > 1000
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
