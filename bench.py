@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle leg")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--rows", type=int, default=None,
+                    help="rows of the 65536 x 8192 workload to use (default: all; smaller slices for tests)")
     return ap.parse_args()
 
 
@@ -188,12 +190,12 @@ def ncu_traffic(kernel: str):
     return float(v) if v else None
 
 
-def make_input(rank: int):
+def make_input(rank: int, rows=None):
     from nvfp4_block_scaled_13_b200 import synth
 
     cfg = synth.CONFIGS[WORKLOAD]
     seed = cfg.seed + 1000 * rank
-    x, shape = synth.make(WORKLOAD, seed=seed)
+    x, shape = synth.make(WORKLOAD, rows=rows, seed=seed)
     return x, shape
 
 
@@ -223,13 +225,13 @@ def run_reference(args, rank, world):
     """--impl reference: the CPU oracle on the machine's host cores (rank 0 only)."""
     if rank != 0:
         return
-    x, (g, r, c) = make_input(0)
+    x, (g, r, c) = make_input(0, args.rows)
     # calibrate, then size each step's sample so that the whole run takes about two minutes
     cal_rows = 64
     t0 = time.perf_counter()
     oracle_step(np.ascontiguousarray(x[: cal_rows * c]), cal_rows, c)
     per_row = (time.perf_counter() - t0) / cal_rows
-    rows = int(max(1, min(4096, 120.0 / max(1, args.steps + args.warmup) / per_row)))
+    rows = int(max(1, min(4096, r // 2, 120.0 / max(1, args.steps + args.warmup) / per_row)))
     for i in range(args.warmup):
         s = (i * rows) % (r - rows)
         oracle_step(np.ascontiguousarray(x[s * c:(s + rows) * c]), rows, c)
@@ -245,7 +247,7 @@ def run_reference(args, rank, world):
         "value": round(value, 6), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": "c5: BF16 65536x8192 (1 GiB) N(0,1), 1% zero blocks, 1% blocks x1e-6; "
+        "config": {"workload": f"c5: BF16 {r}x{c} N(0,1), 1% zero blocks, 1% blocks x1e-6; "
                                "Four Over Six, MSE rule", "shape": [1, r, c], "step": "amax + quantize + dequantize"},
         "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -262,7 +264,7 @@ def run_ours(args, rank, world, local):
     nv.load()
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
-    x_np, (g, r, c) = make_input(rank)
+    x_np, (g, r, c) = make_input(rank, args.rows)
     n, nb = g * r * c, g * r * c // 16
     xd = torch.from_numpy(x_np.view(np.int16)).to(dev)
     amax = torch.empty(g, dtype=torch.float32, device=dev)
@@ -360,7 +362,7 @@ def run_ours(args, rank, world, local):
     # ---- CPU oracle on a bounded sample (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(x_np, c)
+        cpu = cpu_baseline(x_np, c, rows=min(12288, r))
 
     if rank == 0:
         peak, peak_kind = measured_peak()
@@ -373,7 +375,7 @@ def run_ours(args, rank, world, local):
             "ms_per_step": round(step_ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
             "config": {
-                "workload": "c5: BF16 65536x8192 (1 GiB) N(0,1), 1% zero blocks, 1% blocks x1e-6; "
+                "workload": f"c5: BF16 {r}x{c} ({2 * n / 2**30:.3g} GiB) N(0,1), 1% zero blocks, 1% blocks x1e-6; "
                             "Four Over Six, MSE rule; one tensor per rank",
                 "shape": [g, r, c], "step": "amax + quantize (codes, scales, tscale, choice) + dequantize",
                 "l2": "no flush: every step streams 1 GiB of input, 8x the 126 MB L2",

@@ -8,6 +8,15 @@
 // 32-byte vector loads and writes 256 contiguous bytes of codes, 32 bytes of scales and one
 // 32-bit word of choice bits (a warp ballot). Grids are persistent (a multiple of the SM
 // count) and each thread prefetches its next block before working on the current one.
+//
+// The quantizer is issue-bound, not memory-bound, so the per-block arithmetic is kept small:
+//  - block scales without a division: t' = m * RN(1/beta) is within a few ulps of the exact
+//    quotient RN(m/beta), so when E4M3(t' * (1 - 2^-20)) == E4M3(t' * (1 + 2^-20)) the
+//    scale is proven; otherwise (rare) the exact division decides;
+//  - the decode scale d = RN(f32(s) * alpha) and its reciprocal for every E4M3 code s come
+//    from a 128-entry table per group in shared memory (kernels whose CTAs work inside one
+//    group at a time), or are computed per block (the generic kernel);
+//  - packed .f32x2 arithmetic, three-input max, and 32-bit in-group indices.
 #pragma once
 
 #include <float.h>
@@ -21,8 +30,8 @@ constexpr int kThreads = 256;
 
 enum Rule : int { kMaxErr = 0, kMae = 1, kMse = 2 };
 
-// Group lookup: g = b / blocks_per_group. Division by an invariant integer with a
-// precomputed multiplier (exact for b < 2^31); the 64-bit quotient is the fallback.
+// Group lookup for the generic kernel: g = b / blocks_per_group. Division by an invariant
+// integer with a precomputed multiplier (exact for b < 2^31); the 64-bit quotient otherwise.
 struct GroupDiv {
     int64_t bpg;          // blocks per group
     uint32_t mul;         // ceil(2^(31 + l) / bpg), l = ceil(log2 bpg)
@@ -49,6 +58,7 @@ struct QuantParams {
     uint16_t* y;         // fake-quant output or nullptr
     int64_t nblocks;
     int64_t choice_bytes;
+    int64_t groups;
     GroupDiv gdiv;
 };
 
@@ -58,10 +68,163 @@ struct DequantParams {
     const float* tscale;
     uint16_t* y;
     int64_t nblocks;
+    int64_t groups;
     GroupDiv gdiv;
 };
 
-// ---- amax --------------------------------------------------------------------------------
+// ---- small helpers ------------------------------------------------------------------------------
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ float recip_clamped(float d) {
+    return d > 0.0f ? fminf(__frcp_rn(d), FLT_MAX) : 0.0f;
+}
+
+// Per-group constants: alpha = amax / (6 M), beta_K = K * alpha, and the reciprocals of the
+// betas used to bracket the block-scale quotients (valid when both lie in [2^-125, 2^125],
+// so that the reciprocals are normal numbers within half an ulp).
+struct GroupCtx {
+    float alpha, beta6, beta4, y6, y4;
+    bool fast;
+};
+
+template <bool FOUR>
+__device__ __forceinline__ GroupCtx make_group(float amax, float six_m) {
+    GroupCtx c;
+    c.alpha = __fdiv_rn(amax, six_m);
+    c.beta6 = __fmul_rn(6.0f, c.alpha);
+    c.beta4 = __fmul_rn(4.0f, c.alpha);
+    const float lo = FOUR ? c.beta4 : c.beta6;
+    c.fast = lo >= 0x1p-125f && c.beta6 <= 0x1p125f;
+    c.y6 = c.fast ? __frcp_rn(c.beta6) : 0.0f;
+    c.y4 = c.fast ? __frcp_rn(c.beta4) : 0.0f;
+    return c;
+}
+
+// E4M3(RN(m / beta_6)) in the low byte and E4M3(RN(m / beta_4)) in the high byte.
+// t' = RN(m * RN(1/beta)) is within 3 ulps of RN(m / beta); scaling it by 1 -+ 2^-20 gives a
+// bracket that contains RN(m / beta), and E4M3 rounding is monotone, so equal conversions of
+// the two ends are the exact scale. Near a boundary, or outside the bracket's valid range,
+// the exact division decides.
+template <bool FOUR>
+__device__ __forceinline__ uint32_t block_scales(float m, const GroupCtx& c) {
+    if (c.fast) {
+        constexpr float kLo = 1.0f - 0x1p-20f, kHi = 1.0f + 0x1p-20f;
+        const float t6 = __fmul_rn(m, c.y6);
+        const uint32_t b6 = e4m3x2(__fmul_rn(t6, kLo), __fmul_rn(t6, kHi));
+        uint32_t b4 = 0;
+        if (FOUR) {
+            const float t4 = __fmul_rn(m, c.y4);
+            b4 = e4m3x2(__fmul_rn(t4, kLo), __fmul_rn(t4, kHi));
+        }
+        const bool same6 = (b6 & 0xFFu) == (b6 >> 8);
+        const bool same4 = !FOUR || (b4 & 0xFFu) == (b4 >> 8);
+        if (same6 && same4) return (b6 & 0xFFu) | ((b4 & 0xFFu) << 8);
+    }
+    const float t6 = c.beta6 > 0.0f ? __fdiv_rn(m, c.beta6) : 0.0f;
+    const float t4 = FOUR ? (c.beta4 > 0.0f ? __fdiv_rn(m, c.beta4) : 0.0f) : 0.0f;
+    return e4m3x2(t6, t4);
+}
+
+// Decode scale and encode factor for E4M3 code s: d = RN(f32(s) * alpha), r = min(1/d, FLT_MAX).
+__device__ __forceinline__ float2 scale_entry(uint32_t s, float alpha) {
+    const float d = __fmul_rn(e4m3x2_to_float2(s).x, alpha);
+    return make_float2(d, recip_clamped(d));
+}
+
+// One candidate (target maximum K) of one block: its codes, their exact values as f16x2
+// words, and the rule's error. e_i = x_i - v_i * d is one fused multiply-add (the exact
+// difference, rounded once). MAE/MSE keep two running sums, one over even and one over odd
+// element indices (for MSE the two lanes of a packed pair), added at the end.
+template <int RULE>
+__device__ __forceinline__ float candidate(const float2 (&x)[8], float r, float d, uint32_t& c_lo,
+                                           uint32_t& c_hi, uint32_t (&h)[8]) {
+    const float2 rr = make_float2(r, r), nd = make_float2(-d, -d);
+    float2 y[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = mul2(x[j], rr);
+    c_lo = e2m1x8_and_decode(y[0], y[1], y[2], y[3], h[0], h[1], h[2], h[3]);
+    c_hi = e2m1x8_and_decode(y[4], y[5], y[6], y[7], h[4], h[5], h[6], h[7]);
+    float2 acc = make_float2(0.0f, 0.0f);
+    float emax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float2 e = fma2(f16x2_to_float2(h[j]), nd, x[j]);
+        if (RULE == kMse) {
+            acc = fma2(e, e, acc);
+        } else if (RULE == kMae) {
+            acc.x = __fadd_rn(acc.x, fabsf(e.x));
+            acc.y = __fadd_rn(acc.y, fabsf(e.y));
+        } else {
+            emax = max3(emax, fabsf(e.x), fabsf(e.y));
+        }
+    }
+    return RULE == kMaxErr ? emax : __fadd_rn(acc.x, acc.y);
+}
+
+// Quantize the block in `w` (eight BF16 pairs). Stores its codes + scale (or fake-quant
+// BF16) and returns whether target 4 was kept. TABLE: d and 1/d come from `tab`.
+template <bool FOUR, int RULE, bool FQ, bool TABLE>
+__device__ __forceinline__ bool quantize_block(const uint32_t (&w)[8], const GroupCtx& gc, const float2* tab,
+                                               uint8_t* codes8, uint8_t* scale1, uint16_t* y16) {
+    float2 x[8];
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        x[j] = unpack_bf16x2(w[j]);
+        m = max3(m, fabsf(x[j].x), fabsf(x[j].y));
+    }
+    const uint32_t s2 = block_scales<FOUR>(m, gc);
+    const float2 e6 = TABLE ? tab[s2 & 0xFFu] : scale_entry(s2 & 0xFFu, gc.alpha);
+    uint32_t clo, chi, h[8];
+    const float err6 = candidate<RULE>(x, e6.y, e6.x, clo, chi, h);
+    uint32_t s = s2 & 0xFFu;
+    float dsel = e6.x;
+    bool four = false;
+    if (FOUR) {
+        const float2 e4 = TABLE ? tab[s2 >> 8] : scale_entry(s2 >> 8, gc.alpha);
+        uint32_t c4lo, c4hi, h4[8];
+        const float err4 = candidate<RULE>(x, e4.y, e4.x, c4lo, c4hi, h4);
+        four = err4 < err6;   // ties keep target 6
+        if (four) {
+            clo = c4lo;
+            chi = c4hi;
+            s = s2 >> 8;
+            dsel = e4.x;
+        }
+        if (FQ) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) h[j] = four ? h4[j] : h[j];
+        }
+    }
+    if (FQ) {   // q = RN(v * d) of the kept candidate, rounded to BF16
+        const float2 dd = make_float2(dsel, dsel);
+        uint32_t out[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) out[j] = bf16x2(mul2(f16x2_to_float2(h[j]), dd));
+        st32(y16, out);
+    } else {
+        st8(codes8, clo, chi);
+        *scale1 = static_cast<uint8_t>(s);
+    }
+    return four;
+}
+
+// Store one warp's 32 choice bits (the word starting at flat block `first`, a multiple of 32).
+__device__ __forceinline__ void store_choice(uint8_t* choice, int64_t choice_bytes, int64_t first, uint32_t bits) {
+    const int64_t byte0 = first >> 3;
+    if (byte0 + 4 <= choice_bytes) {
+        *reinterpret_cast<uint32_t*>(choice + byte0) = bits;
+    } else {
+        for (int k = 0; byte0 + k < choice_bytes; ++k) choice[byte0 + k] = static_cast<uint8_t>(bits >> (8 * k));
+    }
+}
+
+// ---- amax --------------------------------------------------------------------------------------
 
 // amax[g] = max |x| over group g. BF16 magnitudes compare like their bit patterns, so the
 // reduction runs on (bits & 0x7FFF) as packed unsigned 16-bit pairs; the result's bits
@@ -103,61 +266,73 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
         if (lane == 0) warp_max[warp] = m;
         __syncthreads();
         if (warp == 0) {
-            uint32_t w = lane < kThreads / 32 ? warp_max[lane] : 0u;
-            w = __reduce_max_sync(0xFFFFFFFFu, w);
-            if (lane == 0 && w != 0) atomicMax(reinterpret_cast<unsigned int*>(amax + g), w << 16);
+            uint32_t v = lane < kThreads / 32 ? warp_max[lane] : 0u;
+            v = __reduce_max_sync(0xFFFFFFFFu, v);
+            if (lane == 0 && v != 0) atomicMax(reinterpret_cast<unsigned int*>(amax + g), v << 16);
         }
         __syncthreads();
     }
 }
 
-// ---- quantize / fake-quant -----------------------------------------------------------------
+// ---- quantize / fake-quant: CTAs inside one group at a time (scale table in shared memory) ------
 
-// One candidate (target maximum K) of one block: its codes, their exact values as f16x2
-// words, and the rule's error. e_i = x_i - v_i * d is one fused multiply-add (the exact
-// difference, rounded once). The two running sums of MAE/MSE are the two lanes of a packed
-// pair (even and odd element indices), added at the end.
-template <int RULE>
-__device__ __forceinline__ float candidate(const float2 (&x)[8], float r, float d, uint32_t& c_lo,
-                                           uint32_t& c_hi, uint32_t (&h)[8]) {
-    const float2 rr = make_float2(r, r), nd = make_float2(-d, -d);
-    float2 y[8];
+// Grid: x = CTAs per group, y = groups (looping when there are more than gridDim.y).
+// Requires every group to start on a 32-block boundary of the flat index (one group, or
+// blocks_per_group % 32 == 0) so each warp's 32 choice bits form one aligned word, and
+// blocks_per_group < 2^30.
+template <bool FOUR, int RULE, bool FQ>
+__global__ void __launch_bounds__(kThreads) quantize_grouped_kernel(const QuantParams p) {
+    constexpr float kSixM = FOUR ? 1536.0f : 2688.0f;   // 6 * 256 or 6 * 448
+    __shared__ float2 tab[128];
+    const int lane = threadIdx.x & 31;
+    const uint32_t bpg = static_cast<uint32_t>(p.gdiv.bpg);
+    const uint32_t bpg_pad = (bpg + 31u) & ~31u;
+    const uint32_t stride = gridDim.x * kThreads;
+    for (int64_t g = blockIdx.y; g < p.groups; g += gridDim.y) {
+        const GroupCtx gc = make_group<FOUR>(__ldg(p.amax + g), kSixM);
+        __syncthreads();                       // the previous group's table is no longer read
+        if (threadIdx.x < 128) tab[threadIdx.x] = scale_entry(threadIdx.x == 127 ? 126u : threadIdx.x, gc.alpha);
+        if (!FQ && blockIdx.x == 0 && threadIdx.x == 0) p.tscale[g] = gc.alpha;
+        __syncthreads();
+        const int64_t base = g * static_cast<int64_t>(bpg);
+        const uint16_t* xg = p.x + base * 16;
+        uint8_t* cg = FQ ? nullptr : p.codes + base * 8;
+        uint8_t* sg = FQ ? nullptr : p.scales + base;
+        uint16_t* yg = FQ ? p.y + base * 16 : nullptr;
+        uint32_t lb = blockIdx.x * kThreads + threadIdx.x;
+        uint32_t nxt[8];
+        if (lb < bpg) ld32_stream(xg + static_cast<size_t>(lb) * 16, nxt);
+        for (; lb < bpg_pad; lb += stride) {
+            uint32_t cur[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) y[j] = mul2(x[j], rr);
-    c_lo = e2m1x8_and_decode(y[0], y[1], y[2], y[3], h[0], h[1], h[2], h[3]);
-    c_hi = e2m1x8_and_decode(y[4], y[5], y[6], y[7], h[4], h[5], h[6], h[7]);
-    float2 acc = make_float2(0.0f, 0.0f);
-    float emax = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const float2 e = fma2(f16x2_to_float2(h[j]), nd, x[j]);
-        if (RULE == kMse) {
-            acc = fma2(e, e, acc);
-        } else if (RULE == kMae) {
-            acc = add2(acc, make_float2(fabsf(e.x), fabsf(e.y)));
-        } else {
-            emax = fmaxf(emax, fmaxf(fabsf(e.x), fabsf(e.y)));
+            for (int k = 0; k < 8; ++k) cur[k] = nxt[k];
+            const uint32_t ln = lb + stride;
+            if (ln < bpg) ld32_stream(xg + static_cast<size_t>(ln) * 16, nxt);
+            bool four = false;
+            if (lb < bpg)
+                four = quantize_block<FOUR, RULE, FQ, true>(cur, gc, tab, FQ ? nullptr : cg + static_cast<size_t>(lb) * 8,
+                                                            FQ ? nullptr : sg + lb,
+                                                            FQ ? yg + static_cast<size_t>(lb) * 16 : nullptr);
+            if (p.choice != nullptr) {
+                const uint32_t bits = __ballot_sync(0xFFFFFFFFu, four);
+                if (lane == 0) store_choice(p.choice, p.choice_bytes, base + (lb - lane), bits);
+            }
         }
     }
-    return RULE == kMaxErr ? emax : __fadd_rn(acc.x, acc.y);
 }
 
-__device__ __forceinline__ float recip_clamped(float d) {
-    return d > 0.0f ? fminf(__frcp_rn(d), FLT_MAX) : 0.0f;
-}
+// ---- quantize / fake-quant: flat grid over all blocks (any group layout) ------------------------
 
-// FOUR: Four Over Six (two candidates) or scale-6 (one). FQ: write fake-quant BF16 instead of
-// codes + scales + tensor scale.
 template <bool FOUR, int RULE, bool FQ>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p) {
-    constexpr float kSixM = FOUR ? 1536.0f : 2688.0f;   // 6 * 256 or 6 * 448
+    constexpr float kSixM = FOUR ? 1536.0f : 2688.0f;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
     const int64_t nb_pad = (p.nblocks + 31) & ~int64_t(31);
     const int lane = threadIdx.x & 31;
     int64_t b = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
 
-    int64_t g_start = 0, g_end = 0;
-    float alpha = 0.0f, beta6 = 0.0f, beta4 = 0.0f;
+    int64_t g_end = 0;
+    GroupCtx gc{};
 
     uint32_t nxt[8];
     if (b < p.nblocks) ld32_stream(p.x + b * 16, nxt);
@@ -171,75 +346,26 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p)
 
         bool four = false;
         if (b < p.nblocks) {
-            if (b >= g_end) {   // entering a new group: its tensor scale and the two betas
+            if (b >= g_end) {   // entering a new group
                 const int64_t g = p.gdiv(b);
-                g_start = g * p.gdiv.bpg;
+                const int64_t g_start = g * p.gdiv.bpg;
                 g_end = g_start + p.gdiv.bpg;
-                alpha = __fdiv_rn(__ldg(p.amax + g), kSixM);
-                beta6 = __fmul_rn(6.0f, alpha);
-                beta4 = __fmul_rn(4.0f, alpha);
-                if (!FQ && b == g_start) p.tscale[g] = alpha;
+                gc = make_group<FOUR>(__ldg(p.amax + g), kSixM);
+                if (!FQ && b == g_start) p.tscale[g] = gc.alpha;
             }
-            float2 x[8];
-            float m = 0.0f;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                x[j] = unpack_bf16x2(cur[j]);
-                m = fmaxf(m, fmaxf(fabsf(x[j].x), fabsf(x[j].y)));
-            }
-            // block scales of both candidates with one paired E4M3 conversion
-            const float t6 = beta6 > 0.0f ? __fdiv_rn(m, beta6) : 0.0f;
-            const float t4 = FOUR ? (beta4 > 0.0f ? __fdiv_rn(m, beta4) : 0.0f) : 0.0f;
-            const uint32_t s2 = e4m3x2(t6, t4);
-            const float2 sf = e4m3x2_to_float2(s2);
-            const float d6 = __fmul_rn(sf.x, alpha);
-            uint32_t c6lo, c6hi, h[8];
-            const float err6 = candidate<RULE>(x, recip_clamped(d6), d6, c6lo, c6hi, h);
-            uint32_t clo = c6lo, chi = c6hi, s = s2 & 0xFFu;
-            float dsel = d6;
-            if (FOUR) {
-                const float d4 = __fmul_rn(sf.y, alpha);
-                uint32_t c4lo, c4hi, h4[8];
-                const float err4 = candidate<RULE>(x, recip_clamped(d4), d4, c4lo, c4hi, h4);
-                four = err4 < err6;   // ties keep target 6
-                if (four) {
-                    clo = c4lo;
-                    chi = c4hi;
-                    s = s2 >> 8;
-                    dsel = d4;
-                }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) h[j] = four ? h4[j] : h[j];
-            }
-            if (FQ) {   // q = RN(v * d) of the kept candidate, rounded to BF16
-                const float2 dd = make_float2(dsel, dsel);
-                uint32_t out[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) out[j] = bf16x2(mul2(f16x2_to_float2(h[j]), dd));
-                st32(p.y + b * 16, out);
-            } else {
-                st8(p.codes + b * 8, clo, chi);
-                p.scales[b] = static_cast<uint8_t>(s);
-            }
+            four = quantize_block<FOUR, RULE, FQ, false>(cur, gc, nullptr, FQ ? nullptr : p.codes + b * 8,
+                                                         FQ ? nullptr : p.scales + b, FQ ? p.y + b * 16 : nullptr);
         }
         if (p.choice != nullptr) {
             const uint32_t bits = __ballot_sync(0xFFFFFFFFu, four);
-            if (lane == 0) {
-                const int64_t byte0 = (b - lane) >> 3;   // first block of the warp is a multiple of 32
-                if (byte0 + 4 <= p.choice_bytes) {
-                    *reinterpret_cast<uint32_t*>(p.choice + byte0) = bits;
-                } else {
-                    for (int k = 0; byte0 + k < p.choice_bytes; ++k)
-                        p.choice[byte0 + k] = static_cast<uint8_t>(bits >> (8 * k));
-                }
-            }
+            if (lane == 0) store_choice(p.choice, p.choice_bytes, b - lane, bits);
         }
     }
 }
 
 // ---- dequantize ------------------------------------------------------------------------------
 
-__global__ void __launch_bounds__(kThreads) dequantize_kernel(const DequantParams p) {
+__global__ void __launch_bounds__(kThreads, 4) dequantize_kernel(const DequantParams p) {
     const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
     int64_t b = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
     int64_t g_end = 0;

@@ -102,9 +102,23 @@ nvfp4_status launch_status() {
 
 template <bool FOUR, int RULE, bool FQ>
 nvfp4_status launch_quant(const nvfp4::QuantParams& p, cudaStream_t stream) {
-    auto kernel = nvfp4::quantize_kernel<FOUR, RULE, FQ>;
-    const unsigned grid = grid_for(kernel, p.nblocks);
-    kernel<<<grid, kThreads, 0, stream>>>(p);
+    const int64_t bpg = p.gdiv.bpg;
+    const bool grouped = (p.groups == 1 || bpg % 32 == 0) && bpg < (int64_t(1) << 30);
+    if (grouped) {
+        // CTAs work inside one group at a time, with the group's scale table in shared memory
+        auto kernel = nvfp4::quantize_grouped_kernel<FOUR, RULE, FQ>;
+        const int64_t full = static_cast<int64_t>(sm_count()) * ctas_per_sm(kernel);
+        const int64_t gy = p.groups < 65535 ? p.groups : 65535;
+        int64_t gx = full / gy;
+        const int64_t need = (bpg + kThreads - 1) / kThreads;
+        if (gx > need) gx = need;
+        if (gx < 1) gx = 1;
+        kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), kThreads, 0, stream>>>(p);
+    } else {
+        auto kernel = nvfp4::quantize_kernel<FOUR, RULE, FQ>;
+        const unsigned grid = grid_for(kernel, p.nblocks);
+        kernel<<<grid, kThreads, 0, stream>>>(p);
+    }
     return launch_status();
 }
 
@@ -186,10 +200,8 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t groups, int64_t rows, int
     p.y = nullptr;
     p.nblocks = n / 16;
     p.choice_bytes = (p.nblocks + 7) / 8;
+    p.groups = groups;
     p.gdiv = make_gdiv(groups, rows * cols / 16, p.nblocks);
-    if (mode == NVFP4_SCALE6 && choice != nullptr) {
-        // the kernel's ballot writes zero words; nothing else is needed
-    }
     return dispatch_quant<false>(mode, rule, p, stream);
 }
 
@@ -212,6 +224,7 @@ nvfp4_status nvfp4_fakequant(const uint16_t* x, int64_t groups, int64_t rows, in
     p.y = y;
     p.nblocks = n / 16;
     p.choice_bytes = (p.nblocks + 7) / 8;
+    p.groups = groups;
     p.gdiv = make_gdiv(groups, rows * cols / 16, p.nblocks);
     return dispatch_quant<true>(mode, rule, p, stream);
 }
@@ -230,6 +243,7 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const
     p.tscale = tscale;
     p.y = y;
     p.nblocks = n / 16;
+    p.groups = groups;
     p.gdiv = make_gdiv(groups, rows * cols / 16, p.nblocks);
     const unsigned grid = grid_for(nvfp4::dequantize_kernel, p.nblocks);
     nvfp4::dequantize_kernel<<<grid, kThreads, 0, stream>>>(p);
