@@ -114,16 +114,16 @@ template <bool FOUR>
 __device__ __forceinline__ uint32_t block_scales(float m, const GroupCtx& c) {
     if (c.fast) {
         constexpr float kLo = 1.0f - 0x1p-20f, kHi = 1.0f + 0x1p-20f;
-        const float t6 = __fmul_rn(m, c.y6);
-        const uint32_t b6 = e4m3x2(__fmul_rn(t6, kLo), __fmul_rn(t6, kHi));
-        uint32_t b4 = 0;
         if (FOUR) {
-            const float t4 = __fmul_rn(m, c.y4);
-            b4 = e4m3x2(__fmul_rn(t4, kLo), __fmul_rn(t4, kHi));
+            const float2 t = mul2(make_float2(m, m), make_float2(c.y6, c.y4));
+            const float2 lo = mul2(t, make_float2(kLo, kLo)), hi = mul2(t, make_float2(kHi, kHi));
+            const uint32_t w = e4m3x2(lo.x, hi.x) | (e4m3x2(lo.y, hi.y) << 16);   // lo6 hi6 lo4 hi4
+            if (((w ^ (w >> 8)) & 0x00FF00FFu) == 0u) return __byte_perm(w, 0u, 0x4420);
+        } else {
+            const float t6 = __fmul_rn(m, c.y6);
+            const uint32_t b6 = e4m3x2(__fmul_rn(t6, kLo), __fmul_rn(t6, kHi));
+            if ((b6 & 0xFFu) == (b6 >> 8)) return b6 & 0xFFu;
         }
-        const bool same6 = (b6 & 0xFFu) == (b6 >> 8);
-        const bool same4 = !FOUR || (b4 & 0xFFu) == (b4 >> 8);
-        if (same6 && same4) return (b6 & 0xFFu) | ((b4 & 0xFFu) << 8);
     }
     const float t6 = c.beta6 > 0.0f ? __fdiv_rn(m, c.beta6) : 0.0f;
     const float t4 = FOUR ? (c.beta4 > 0.0f ? __fdiv_rn(m, c.beta4) : 0.0f) : 0.0f;
@@ -277,17 +277,22 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
 // ---- quantize / fake-quant: CTAs inside one group at a time (scale table in shared memory) ------
 
 // Grid: x = CTAs per group, y = groups (looping when there are more than gridDim.y).
+// Each warp works on tiles of 64 consecutive blocks of its group: lane t quantizes blocks t and
+// t + 32 of the tile, so both 32-byte loads, both code stores and both scale stores of a warp
+// are contiguous, and each half-tile's 32 choice bits are one ballot word. The next tile's two
+// blocks are loaded before the current ones are worked on.
 // Requires every group to start on a 32-block boundary of the flat index (one group, or
-// blocks_per_group % 32 == 0) so each warp's 32 choice bits form one aligned word, and
-// blocks_per_group < 2^30.
+// blocks_per_group % 32 == 0) and blocks_per_group < 2^30.
 template <bool FOUR, int RULE, bool FQ>
-__global__ void __launch_bounds__(kThreads) quantize_grouped_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kernel(const QuantParams p) {
     constexpr float kSixM = FOUR ? 1536.0f : 2688.0f;   // 6 * 256 or 6 * 448
     __shared__ float2 tab[128];
-    const int lane = threadIdx.x & 31;
+    const uint32_t lane = threadIdx.x & 31u;
     const uint32_t bpg = static_cast<uint32_t>(p.gdiv.bpg);
-    const uint32_t bpg_pad = (bpg + 31u) & ~31u;
-    const uint32_t stride = gridDim.x * kThreads;
+    const uint32_t ntiles = (bpg + 63u) >> 6;
+    const uint32_t warps = gridDim.x * (kThreads / 32);
+    const uint32_t warp0 = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    const int64_t choice_words = p.choice_bytes >> 2;          // whole 32-bit words of the bitmap
     for (int64_t g = blockIdx.y; g < p.groups; g += gridDim.y) {
         const GroupCtx gc = make_group<FOUR>(__ldg(p.amax + g), kSixM);
         __syncthreads();                       // the previous group's table is no longer read
@@ -299,23 +304,56 @@ __global__ void __launch_bounds__(kThreads) quantize_grouped_kernel(const QuantP
         uint8_t* cg = FQ ? nullptr : p.codes + base * 8;
         uint8_t* sg = FQ ? nullptr : p.scales + base;
         uint16_t* yg = FQ ? p.y + base * 16 : nullptr;
-        uint32_t lb = blockIdx.x * kThreads + threadIdx.x;
-        uint32_t nxt[8];
-        if (lb < bpg) ld32_stream(xg + static_cast<size_t>(lb) * 16, nxt);
-        for (; lb < bpg_pad; lb += stride) {
-            uint32_t cur[8];
+        uint32_t* chw = reinterpret_cast<uint32_t*>(p.choice) + (base >> 5);   // base is a multiple of 32
+        const int64_t chw_left = choice_words - (base >> 5);
+        uint32_t tile = warp0;
+        uint32_t na[8], nb[8];
+        {
+            const uint32_t a = (tile << 6) + lane;
+            if (tile < ntiles && a < bpg) ld32_stream(xg + static_cast<size_t>(a) * 16, na);
+            if (tile < ntiles && a + 32u < bpg) ld32_stream(xg + static_cast<size_t>(a + 32u) * 16, nb);
+        }
+        for (; tile < ntiles; tile += warps) {
+            uint32_t ca[8], cb[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) cur[k] = nxt[k];
-            const uint32_t ln = lb + stride;
-            if (ln < bpg) ld32_stream(xg + static_cast<size_t>(ln) * 16, nxt);
-            bool four = false;
-            if (lb < bpg)
-                four = quantize_block<FOUR, RULE, FQ, true>(cur, gc, tab, FQ ? nullptr : cg + static_cast<size_t>(lb) * 8,
-                                                            FQ ? nullptr : sg + lb,
-                                                            FQ ? yg + static_cast<size_t>(lb) * 16 : nullptr);
+            for (int k = 0; k < 8; ++k) {
+                ca[k] = na[k];
+                cb[k] = nb[k];
+            }
+            const uint32_t a = (tile << 6) + lane;
+            const uint32_t an = ((tile + warps) << 6) + lane;
+            if (tile + warps < ntiles) {
+                if (an < bpg) ld32_stream(xg + static_cast<size_t>(an) * 16, na);
+                if (an + 32u < bpg) ld32_stream(xg + static_cast<size_t>(an + 32u) * 16, nb);
+            }
+            bool fa = false, fb = false;
+            if ((tile << 6) + 64u <= bpg) {    // interior tile: all 64 blocks exist (warp-uniform)
+                fa = quantize_block<FOUR, RULE, FQ, true>(ca, gc, tab, FQ ? nullptr : cg + static_cast<size_t>(a) * 8,
+                                                          FQ ? nullptr : sg + a, FQ ? yg + static_cast<size_t>(a) * 16 : nullptr);
+                fb = quantize_block<FOUR, RULE, FQ, true>(cb, gc, tab, FQ ? nullptr : cg + static_cast<size_t>(a + 32u) * 8,
+                                                          FQ ? nullptr : sg + a + 32u,
+                                                          FQ ? yg + static_cast<size_t>(a + 32u) * 16 : nullptr);
+            } else {
+                if (a < bpg)
+                    fa = quantize_block<FOUR, RULE, FQ, true>(ca, gc, tab, FQ ? nullptr : cg + static_cast<size_t>(a) * 8,
+                                                              FQ ? nullptr : sg + a,
+                                                              FQ ? yg + static_cast<size_t>(a) * 16 : nullptr);
+                if (a + 32u < bpg)
+                    fb = quantize_block<FOUR, RULE, FQ, true>(cb, gc, tab,
+                                                              FQ ? nullptr : cg + static_cast<size_t>(a + 32u) * 8,
+                                                              FQ ? nullptr : sg + a + 32u,
+                                                              FQ ? yg + static_cast<size_t>(a + 32u) * 16 : nullptr);
+            }
             if (p.choice != nullptr) {
-                const uint32_t bits = __ballot_sync(0xFFFFFFFFu, four);
-                if (lane == 0) store_choice(p.choice, p.choice_bytes, base + (lb - lane), bits);
+                const uint32_t bits_a = __ballot_sync(0xFFFFFFFFu, fa);
+                const uint32_t bits_b = __ballot_sync(0xFFFFFFFFu, fb);
+                // lane 0 stores the word of blocks [64 tile, +32), lane 1 the next one (if any)
+                const uint32_t w = 2u * tile + lane;
+                if (lane < 2u && (w << 5) < bpg) {
+                    const uint32_t bits = lane ? bits_b : bits_a;
+                    if (static_cast<int64_t>(w) < chw_left) chw[w] = bits;
+                    else store_choice(p.choice, p.choice_bytes, base + (static_cast<int64_t>(w) << 5), bits);
+                }
             }
         }
     }
