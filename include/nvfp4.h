@@ -140,6 +140,23 @@ NVFP4_API nvfp4_status nvfp4_fakequant(const uint16_t* x, int64_t groups, int64_
                              const float* amax, nvfp4_mode mode, nvfp4_rule rule,
                              uint16_t* y, uint8_t* choice, cudaStream_t stream);
 
+/* Quantize a [rows, cols] BF16 matrix for a Blackwell block-scaled FP4 tensor-core GEMM, in
+ * which it is the K-major operand (cols = K). NVFP4 weights and activations are run on
+ * Blackwell's native FP4 tensor cores ("NVIDIA Model Optimizerを用いたNemotron 3.5 Lightning
+ * NVFP4とQADの開発", section on Nemotron 3.5 Lightning and NVFP4; "Nemotron-3 Nano NVFP4" blog
+ * §2). Same arithmetic, codes, tensor scale and choice bits as nvfp4_quantize with one group;
+ * only the scale layout differs: the scales of row r, block column c (c = k / 16) are stored
+ * in tiles of 128 rows x 4 block columns, 512 bytes each, tile (r / 128, c / 4) at byte
+ * ((r / 128) * ceil(cols / 64) + c / 4) * 512, and inside the tile at byte
+ * (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4 (the tiled 1-D block-scaling layout of cuBLASLt).
+ *   scales  [roundup(rows, 128) * roundup(cols / 16, 4)] bytes; the padding is zero-filled
+ *           (one cudaMemsetAsync before the kernel)                                    (out)
+ * rows * cols / 16 must be below 2^30 (else NVFP4_ERR_SHAPE). The library has no counterpart
+ * on the pages for the layout itself; it is the operand format of the FP4 GEMMs they run. */
+NVFP4_API nvfp4_status nvfp4_quantize_gemm(const uint16_t* x, int64_t rows, int64_t cols, const float* amax,
+                                           nvfp4_mode mode, nvfp4_rule rule, uint8_t* codes, uint8_t* scales,
+                                           float* tscale, uint8_t* choice, cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 NVFP4_API const char* nvfp4_status_string(nvfp4_status status);
 

@@ -22,9 +22,9 @@ from typing import NamedTuple
 __all__ = [
     "load", "library_path", "Nvfp4Error",
     "SCALE6", "FOUR_OVER_SIX", "RULE_MAXERR", "RULE_MAE", "RULE_MSE",
-    "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fakequant",
+    "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_quantize_gemm",
     "nvfp4_status_string", "nvfp4_version",
-    "Quantized", "amax", "quantize", "fakequant", "dequantize",
+    "Quantized", "amax", "quantize", "fakequant", "dequantize", "quantize_for_gemm", "gemm_scale_bytes",
 ]
 
 SCALE6, FOUR_OVER_SIX = 0, 1
@@ -60,7 +60,8 @@ def load():
         L.nvfp4_quantize.argtypes = [vp, i64, i64, i64, vp, i32, i32, vp, vp, vp, vp, vp]
         L.nvfp4_dequantize.argtypes = [vp, vp, vp, i64, i64, i64, vp, vp]
         L.nvfp4_fakequant.argtypes = [vp, i64, i64, i64, vp, i32, i32, vp, vp, vp]
-        for f in (L.nvfp4_amax, L.nvfp4_quantize, L.nvfp4_dequantize, L.nvfp4_fakequant):
+        L.nvfp4_quantize_gemm.argtypes = [vp, i64, i64, vp, i32, i32, vp, vp, vp, vp, vp]
+        for f in (L.nvfp4_amax, L.nvfp4_quantize, L.nvfp4_dequantize, L.nvfp4_fakequant, L.nvfp4_quantize_gemm):
             f.restype = i32
         L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
         L.nvfp4_version.argtypes, L.nvfp4_version.restype = [], i32
@@ -126,6 +127,12 @@ def nvfp4_dequantize(codes, scales, tscale, groups, rows, cols, y, stream=None):
 def nvfp4_fakequant(x, groups, rows, cols, amax, mode, rule, y, choice=None, stream=None):
     _check(load().nvfp4_fakequant(_ptr(x), groups, rows, cols, _ptr(amax), _mode(mode), _rule(rule),
                                   _ptr(y), _ptr(choice), _stream(stream)), "nvfp4_fakequant")
+
+
+def nvfp4_quantize_gemm(x, rows, cols, amax, mode, rule, codes, scales, tscale, choice=None, stream=None):
+    _check(load().nvfp4_quantize_gemm(_ptr(x), rows, cols, _ptr(amax), _mode(mode), _rule(rule), _ptr(codes),
+                                      _ptr(scales), _ptr(tscale), _ptr(choice), _stream(stream)),
+           "nvfp4_quantize_gemm")
 
 
 def nvfp4_status_string(status: int) -> str:
@@ -205,3 +212,28 @@ def fakequant(x, mode="four_over_six", rule="mse", groups: int = 1, amax_values=
         out = torch.empty_like(x, dtype=torch.bfloat16)
     nvfp4_fakequant(x, g, r, c, amax_values, mode, rule, out, choice, stream)
     return out
+
+
+def gemm_scale_bytes(rows: int, cols: int) -> int:
+    """Size of the tiled scale buffer of nvfp4_quantize_gemm: roundup(rows, 128) * roundup(cols / 16, 4)."""
+    return (rows + 127) // 128 * 128 * ((cols // 16 + 3) // 4 * 4)
+
+
+def quantize_for_gemm(x, mode="four_over_six", rule="mse", amax_values=None, with_choice=False, stream=None):
+    """Quantize a 2-D BF16 matrix as a K-major block-scaled FP4 GEMM operand. Returns
+    (codes [rows, cols/2] uint8, tiled scales uint8, tscale [1] float32, choice or None)."""
+    import torch
+
+    if x.dim() != 2:
+        raise ValueError("quantize_for_gemm: x must be 2-D [rows, cols]")
+    rows, cols = x.shape
+    if amax_values is None:
+        amax_values = amax(x, 1, stream)
+    dev = x.device
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(gemm_scale_bytes(rows, cols), dtype=torch.uint8, device=dev)
+    tscale = torch.empty(1, dtype=torch.float32, device=dev)
+    nb = rows * cols // 16
+    choice = torch.empty(max(1, (nb + 7) // 8), dtype=torch.uint8, device=dev) if with_choice else None
+    nvfp4_quantize_gemm(x, rows, cols, amax_values, mode, rule, codes, scales, tscale, choice, stream)
+    return codes, scales, tscale, choice

@@ -60,6 +60,9 @@ struct QuantParams {
     int64_t choice_bytes;
     int64_t groups;
     GroupDiv gdiv;
+    // tiled scale layout of block-scaled GEMM operands (one group, a [rows, 16 * bpr] matrix):
+    // blocks per row, multiply-shift divisor for it (exact below 2^31), 4-column tiles per row
+    uint32_t bpr, bpr_mul, bpr_shift, n_ct;
 };
 
 struct DequantParams {
@@ -214,6 +217,15 @@ __device__ __forceinline__ bool quantize_block(const uint32_t (&w)[8], const Gro
     return four;
 }
 
+// Byte offset of local block a's scale in the tiled layout: 128-row x 4-column tiles of 512
+// bytes, tile (row / 128, col / 4) at ((row / 128) * n_ct + col / 4) * 512, and inside a tile
+// row r, column c at (r % 32) * 16 + (r / 32) * 4 + c.
+__device__ __forceinline__ uint32_t tiled_scale_offset(uint32_t a, const QuantParams& p) {
+    const uint32_t row = p.bpr == 1u ? a : __umulhi(a, p.bpr_mul) >> p.bpr_shift;
+    const uint32_t col = a - row * p.bpr;
+    return (((row >> 7) * p.n_ct + (col >> 2)) << 9) + ((row & 31u) << 4) + (((row >> 5) & 3u) << 2) + (col & 3u);
+}
+
 // Store one warp's 32 choice bits (the word starting at flat block `first`, a multiple of 32).
 __device__ __forceinline__ void store_choice(uint8_t* choice, int64_t choice_bytes, int64_t first, uint32_t bits) {
     const int64_t byte0 = first >> 3;
@@ -283,7 +295,8 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
 // blocks are loaded before the current ones are worked on.
 // Requires every group to start on a 32-block boundary of the flat index (one group, or
 // blocks_per_group % 32 == 0) and blocks_per_group < 2^30.
-template <bool FOUR, int RULE, bool FQ>
+// SWZ: scales go to the tiled GEMM layout (one group only).
+template <bool FOUR, int RULE, bool FQ, bool SWZ = false>
 __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kernel(const QuantParams p) {
     constexpr float kSixM = FOUR ? 1536.0f : 2688.0f;   // 6 * 256 or 6 * 448
     __shared__ float2 tab[128];
@@ -329,19 +342,20 @@ __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kerne
             bool fa = false, fb = false;
             if ((tile << 6) + 64u <= bpg) {    // interior tile: all 64 blocks exist (warp-uniform)
                 fa = quantize_block<FOUR, RULE, FQ, true>(ca, gc, tab, FQ ? nullptr : cg + static_cast<size_t>(a) * 8,
-                                                          FQ ? nullptr : sg + a, FQ ? yg + static_cast<size_t>(a) * 16 : nullptr);
+                                                          FQ ? nullptr : (SWZ ? p.scales + tiled_scale_offset(a, p) : sg + a),
+                                                          FQ ? yg + static_cast<size_t>(a) * 16 : nullptr);
                 fb = quantize_block<FOUR, RULE, FQ, true>(cb, gc, tab, FQ ? nullptr : cg + static_cast<size_t>(a + 32u) * 8,
-                                                          FQ ? nullptr : sg + a + 32u,
+                                                          FQ ? nullptr : (SWZ ? p.scales + tiled_scale_offset(a + 32u, p) : sg + a + 32u),
                                                           FQ ? yg + static_cast<size_t>(a + 32u) * 16 : nullptr);
             } else {
                 if (a < bpg)
                     fa = quantize_block<FOUR, RULE, FQ, true>(ca, gc, tab, FQ ? nullptr : cg + static_cast<size_t>(a) * 8,
-                                                              FQ ? nullptr : sg + a,
+                                                              FQ ? nullptr : (SWZ ? p.scales + tiled_scale_offset(a, p) : sg + a),
                                                               FQ ? yg + static_cast<size_t>(a) * 16 : nullptr);
                 if (a + 32u < bpg)
                     fb = quantize_block<FOUR, RULE, FQ, true>(cb, gc, tab,
                                                               FQ ? nullptr : cg + static_cast<size_t>(a + 32u) * 8,
-                                                              FQ ? nullptr : sg + a + 32u,
+                                                              FQ ? nullptr : (SWZ ? p.scales + tiled_scale_offset(a + 32u, p) : sg + a + 32u),
                                                               FQ ? yg + static_cast<size_t>(a + 32u) * 16 : nullptr);
             }
             if (p.choice != nullptr) {

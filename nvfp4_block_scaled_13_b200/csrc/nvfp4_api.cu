@@ -132,6 +132,27 @@ nvfp4_status dispatch_quant(nvfp4_mode mode, nvfp4_rule rule, const nvfp4::Quant
     }
 }
 
+template <bool FOUR, int RULE>
+nvfp4_status launch_quant_gemm(const nvfp4::QuantParams& p, cudaStream_t stream) {
+    auto kernel = nvfp4::quantize_grouped_kernel<FOUR, RULE, false, true>;
+    const int64_t full = static_cast<int64_t>(sm_count()) * ctas_per_sm(kernel);
+    int64_t gx = full;
+    const int64_t need = (p.nblocks + kThreads - 1) / kThreads;
+    if (gx > need) gx = need;
+    if (gx < 1) gx = 1;
+    kernel<<<dim3(static_cast<unsigned>(gx), 1u), kThreads, 0, stream>>>(p);
+    return launch_status();
+}
+
+nvfp4_status dispatch_quant_gemm(nvfp4_mode mode, nvfp4_rule rule, const nvfp4::QuantParams& p, cudaStream_t s) {
+    if (mode == NVFP4_SCALE6) return launch_quant_gemm<false, nvfp4::kMse>(p, s);
+    switch (rule) {
+        case NVFP4_RULE_MAXERR: return launch_quant_gemm<true, nvfp4::kMaxErr>(p, s);
+        case NVFP4_RULE_MAE: return launch_quant_gemm<true, nvfp4::kMae>(p, s);
+        default: return launch_quant_gemm<true, nvfp4::kMse>(p, s);
+    }
+}
+
 nvfp4_status check_mode_rule(nvfp4_mode mode, nvfp4_rule rule) {
     if (mode != NVFP4_SCALE6 && mode != NVFP4_FOUR_OVER_SIX) return NVFP4_ERR_MODE;
     if (mode == NVFP4_FOUR_OVER_SIX && rule != NVFP4_RULE_MAXERR && rule != NVFP4_RULE_MAE && rule != NVFP4_RULE_MSE)
@@ -248,6 +269,52 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const
     const unsigned grid = grid_for(nvfp4::dequantize_kernel, p.nblocks);
     nvfp4::dequantize_kernel<<<grid, kThreads, 0, stream>>>(p);
     return launch_status();
+}
+
+nvfp4_status nvfp4_quantize_gemm(const uint16_t* x, int64_t rows, int64_t cols, const float* amax, nvfp4_mode mode,
+                                 nvfp4_rule rule, uint8_t* codes, uint8_t* scales, float* tscale, uint8_t* choice,
+                                 cudaStream_t stream) {
+    if (amax == nullptr || tscale == nullptr) return NVFP4_ERR_NULL;
+    int64_t n = 0;
+    nvfp4_status st = check_shape(1, rows, cols, &n);
+    if (st != NVFP4_OK) return st;
+    if (n / 16 >= (int64_t(1) << 30)) return NVFP4_ERR_SHAPE;
+    if (n > 0 && (x == nullptr || codes == nullptr || scales == nullptr)) return NVFP4_ERR_NULL;
+    st = check_mode_rule(mode, rule);
+    if (st != NVFP4_OK) return st;
+    if (!aligned(amax, 4) || !aligned(tscale, 4) || (choice && !aligned(choice, 4))) return NVFP4_ERR_ALIGN;
+    if (n > 0 && (!aligned(x, 32) || !aligned(codes, 8))) return NVFP4_ERR_ALIGN;
+    if (n == 0) {
+        const float six_m = mode == NVFP4_FOUR_OVER_SIX ? 1536.0f : 2688.0f;
+        tensor_scale_only_kernel<<<1, kThreads, 0, stream>>>(amax, tscale, 1, six_m);
+        return launch_status();
+    }
+    const int64_t bpr = cols / 16;
+    const int64_t n_ct = (bpr + 3) / 4;
+    const int64_t padded = (rows + 127) / 128 * 128 * n_ct * 4;
+    if (cudaMemsetAsync(scales, 0, static_cast<size_t>(padded), stream) != cudaSuccess) return NVFP4_ERR_CUDA;
+    nvfp4::QuantParams p{};
+    p.x = x;
+    p.amax = amax;
+    p.codes = codes;
+    p.scales = scales;
+    p.tscale = tscale;
+    p.choice = choice;
+    p.nblocks = n / 16;
+    p.choice_bytes = (p.nblocks + 7) / 8;
+    p.groups = 1;
+    p.gdiv = make_gdiv(1, p.nblocks, p.nblocks);
+    p.bpr = static_cast<uint32_t>(bpr);
+    p.n_ct = static_cast<uint32_t>(n_ct);
+    if (bpr > 1) {
+        // row = floor(a * m / 2^(31 + l)), m = ceil(2^(31 + l) / bpr), l = ceil(log2 bpr): exact for a < 2^31
+        uint32_t l = 0;
+        while ((int64_t(1) << l) < bpr) ++l;
+        const unsigned __int128 num = (unsigned __int128)1 << (31 + l);
+        p.bpr_mul = static_cast<uint32_t>((num + bpr - 1) / bpr);
+        p.bpr_shift = l - 1;
+    }
+    return dispatch_quant_gemm(mode, rule, p, stream);
 }
 
 const char* nvfp4_status_string(nvfp4_status status) {

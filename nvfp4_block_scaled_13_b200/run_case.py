@@ -29,6 +29,7 @@ def main():
     ap.add_argument("--rule", default="mse")
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--fakequant", action="store_true")
+    ap.add_argument("--gemm-layout", action="store_true", help="nvfp4_quantize_gemm (tiled scales; one group)")
     a = ap.parse_args()
 
     nv.load()
@@ -37,7 +38,7 @@ def main():
     xd = torch.from_numpy(x.view(np.int16)).cuda()
     amax = torch.empty(g, dtype=torch.float32, device="cuda")
     codes = torch.empty(n // 2, dtype=torch.uint8, device="cuda")
-    scales = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(nv.gemm_scale_bytes(g * r, c) if a.gemm_layout else nb, dtype=torch.uint8, device="cuda")
     tscale = torch.empty(g, dtype=torch.float32, device="cuda")
     choice = torch.empty((nb + 7) // 8, dtype=torch.uint8, device="cuda")
     y = torch.empty(n, dtype=torch.int16, device="cuda")
@@ -48,14 +49,18 @@ def main():
         ev[1].record()
         if a.fakequant:
             nv.nvfp4_fakequant(xd, g, r, c, amax, a.mode, a.rule, y, choice)
+        elif a.gemm_layout:
+            nv.nvfp4_quantize_gemm(xd, g * r, c, amax, a.mode, a.rule, codes, scales, tscale, choice)
         else:
             nv.nvfp4_quantize(xd, g, r, c, amax, a.mode, a.rule, codes, scales, tscale, choice)
         ev[2].record()
-        nv.nvfp4_dequantize(codes, scales, tscale, g, r, c, y)
+        if not a.gemm_layout:
+            nv.nvfp4_dequantize(codes, scales, tscale, g, r, c, y)
         ev[3].record()
     torch.cuda.synchronize()
     print(f"{a.workload} [{g},{r},{c}] {a.mode}/{a.rule}: amax {ev[0].elapsed_time(ev[1]):.4f} ms, "
-          f"{'fakequant' if a.fakequant else 'quantize'} {ev[1].elapsed_time(ev[2]):.4f} ms, "
+          f"{'fakequant' if a.fakequant else ('quantize_gemm' if a.gemm_layout else 'quantize')} "
+          f"{ev[1].elapsed_time(ev[2]):.4f} ms, "
           f"dequantize {ev[2].elapsed_time(ev[3]):.4f} ms (last rep)")
 
 

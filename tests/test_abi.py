@@ -20,7 +20,7 @@ def header_functions(path):
 def test_header_declares_the_boundary():
     names = header_functions(os.path.join(ROOT, "include", "nvfp4.h"))
     assert names == ["nvfp4_amax", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_quantize",
-                     "nvfp4_status_string", "nvfp4_version"]
+                     "nvfp4_quantize_gemm", "nvfp4_status_string", "nvfp4_version"]
 
 
 def test_library_exports_every_declared_symbol():
@@ -68,6 +68,14 @@ A = 1 << 20          # 32-byte aligned
     (lambda L: L.nvfp4_dequantize(A, A, A, 1, 4, 32, None, None), 1),
     (lambda L: L.nvfp4_dequantize(A, A, A, 1, 4, 31, A, None), 2),
     (lambda L: L.nvfp4_dequantize(A, A, A, 1, 4, 32, A + 8, None), 3),
+    # nvfp4_quantize_gemm(x, R, C, amax, mode, rule, codes, scales, tscale, choice, stream)
+    (lambda L: L.nvfp4_quantize_gemm(A, 4, 32, None, 1, 2, A, A, A, None, None), 1),
+    (lambda L: L.nvfp4_quantize_gemm(A, 4, 32, A, 1, 2, A, None, A, None, None), 1),
+    (lambda L: L.nvfp4_quantize_gemm(A, 4, 40, A, 1, 2, A, A, A, None, None), 2),
+    (lambda L: L.nvfp4_quantize_gemm(A, 1 << 20, 1 << 15, A, 1, 2, A, A, A, None, None), 2),
+    (lambda L: L.nvfp4_quantize_gemm(A, 4, 32, A, 3, 2, A, A, A, None, None), 4),
+    (lambda L: L.nvfp4_quantize_gemm(A, 4, 32, A, 1, 7, A, A, A, None, None), 5),
+    (lambda L: L.nvfp4_quantize_gemm(A + 8, 4, 32, A, 1, 2, A, A, A, None, None), 3),
     # nvfp4_fakequant(x, G, R, C, amax, mode, rule, y, choice, stream)
     (lambda L: L.nvfp4_fakequant(A, 1, 4, 32, A, 1, 2, None, None, None), 1),
     (lambda L: L.nvfp4_fakequant(A, 1, 4, 32, A, 7, 2, A, None, None), 4),
