@@ -51,6 +51,8 @@ def lib():
         L.nvo_e2m1_to_f32.argtypes, L.nvo_e2m1_to_f32.restype = [u8], f32
         for name in ("nvo_f32_to_e2m1_array", "nvo_f32_to_e4m3_array", "nvo_f32_to_bf16_array"):
             getattr(L, name).argtypes, getattr(L, name).restype = [vp, vp, i64], None
+        L.nvo_qad_kl.argtypes = [vp, vp, i64, i64, ctypes.c_double, ctypes.c_double, vp, vp]
+        L.nvo_qad_kl.restype = None
         L.nvo_block_candidate.argtypes = [vp, f32, f32, i32, ctypes.POINTER(Candidate)]
         L.nvo_block_candidate.restype = None
         L.nvo_amax.argtypes, L.nvo_amax.restype = [vp, i64, i64, i64, vp], None
@@ -196,3 +198,15 @@ def dequantize(codes, scales, tscale, groups, rows, cols):
 
 def library_path() -> str:
     return _build.LIB if os.path.exists(_build.LIB) else _build.build()
+
+
+def qad_kl(teacher: np.ndarray, student: np.ndarray, rows: int, vocab: int, tau: float = 1.0,
+           grad_scale: float = 1.0, with_grad: bool = True):
+    """Per-row KL(softmax(teacher/tau) || softmax(student/tau)) and grad_scale * (q - p), binary64."""
+    t = np.ascontiguousarray(teacher, dtype=np.uint16)
+    s = np.ascontiguousarray(student, dtype=np.uint16)
+    assert t.size == rows * vocab and s.size == rows * vocab
+    kl = np.zeros(rows, np.float64)
+    g = np.zeros(rows * vocab, np.float64) if with_grad else None
+    lib().nvo_qad_kl(_ptr(t), _ptr(s), rows, vocab, float(tau), float(grad_scale), _ptr(kl), _ptr(g))
+    return kl, g

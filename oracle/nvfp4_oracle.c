@@ -278,3 +278,35 @@ void nvo_dequantize(const uint8_t* codes, const uint8_t* scales, const float* ts
         }
     }
 }
+
+/* ---- QAD distillation loss (see the header) -------------------------------------------- */
+
+void nvo_qad_kl(const uint16_t* teacher, const uint16_t* student, int64_t rows, int64_t vocab, double tau,
+                double grad_scale, double* kl, double* grad) {
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t* t = teacher + r * vocab;
+        const uint16_t* s = student + r * vocab;
+        /* log-sum-exp of each row, shifted by its maximum */
+        double mt = -INFINITY, ms = -INFINITY;
+        for (int64_t v = 0; v < vocab; ++v) {
+            double a = nvo_bf16_to_f32(t[v]) / tau, b = nvo_bf16_to_f32(s[v]) / tau;
+            if (a > mt) mt = a;
+            if (b > ms) ms = b;
+        }
+        double zt = 0.0, zs = 0.0;
+        for (int64_t v = 0; v < vocab; ++v) {
+            zt += exp(nvo_bf16_to_f32(t[v]) / tau - mt);
+            zs += exp(nvo_bf16_to_f32(s[v]) / tau - ms);
+        }
+        double lse_t = mt + log(zt), lse_s = ms + log(zs);
+        double acc = 0.0;
+        for (int64_t v = 0; v < vocab; ++v) {
+            double a = nvo_bf16_to_f32(t[v]) / tau, b = nvo_bf16_to_f32(s[v]) / tau;
+            double logp = a - lse_t, logq = b - lse_s;
+            double p = exp(logp), q = exp(logq);
+            acc += p * (logp - logq);
+            if (grad) grad[r * vocab + v] = grad_scale * (q - p);
+        }
+        kl[r] = acc;
+    }
+}

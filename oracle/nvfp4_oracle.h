@@ -113,6 +113,19 @@ void nvo_quantize_ex(const uint16_t* x, int64_t groups, int64_t rows, int64_t co
 void nvo_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tscale,
                     int64_t groups, int64_t rows, int64_t cols, uint16_t* y);
 
+/* ---- QAD distillation loss ---------------------------------------------------------------
+ * "Quantization-Aware Distillation for NVFP4 Inference Accuracy Recovery", technical summary
+ * §2 (method): the student (NVFP4, run through simulated quantization) is trained to match
+ * the frozen BF16 teacher's output distribution, loss L = D_KL(p_teacher || p_student).
+ * Per row r of [rows, vocab] BF16 logits, with temperature tau:
+ *   p = softmax(teacher / tau), q = softmax(student / tau),
+ *   kl[r] = sum_v p_v (log p_v - log q_v)                      (natural log, binary64)
+ *   grad[r, v] = grad_scale * (q_v - p_v)   (d kl / d student_v = (q_v - p_v) / tau; the
+ *                                            caller folds 1/tau and any mean into grad_scale)
+ * grad may be NULL. Everything is computed in binary64 from the BF16 inputs. */
+void nvo_qad_kl(const uint16_t* teacher, const uint16_t* student, int64_t rows, int64_t vocab, double tau,
+                double grad_scale, double* kl, double* grad);
+
 #ifdef __cplusplus
 }
 #endif

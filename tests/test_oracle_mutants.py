@@ -34,6 +34,10 @@ MUTANTS = {
     "error_against_scaled_values": ("c->e[i] = fmaf(-v, c->d, x[i]);", "c->e[i] = y - v;"),
     "error_drops_scale": ("c->e[i] = fmaf(-v, c->d, x[i]);", "c->e[i] = x[i] - v;"),
     "zero_sign_dropped": ("uint8_t sign = signbit(y) ? 0x8u : 0x0u;", "uint8_t sign = (y < 0) ? 0x8u : 0x0u;"),
+    "kl_reversed": ("acc += p * (logp - logq);", "acc += q * (logq - logp);"),
+    "kl_grad_sign": ("grad[r * vocab + v] = grad_scale * (q - p);", "grad[r * vocab + v] = grad_scale * (p - q);"),
+    "kl_student_normalizer_dropped": ("double logp = a - lse_t, logq = b - lse_s;", "double logp = a - lse_t, logq = b - ms;"),
+    "kl_tau_on_teacher_only": ("zs += exp(nvo_bf16_to_f32(s[v]) / tau - ms);", "zs += exp(nvo_bf16_to_f32(s[v]) - ms);"),
 }
 
 
@@ -50,6 +54,7 @@ def test_pins_reject_mutant(name, tmp_path):
                     "-I", hdr, str(mut), "-o", str(lib), "-lm"], check=True)
     env = dict(os.environ, NVO_ORACLE_LIB=str(lib))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_qad_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins accepted mutant {name}:\n{r.stdout[-2000:]}"
