@@ -75,7 +75,8 @@ typedef enum {
     NVFP4_ERR_ALIGN = 3,   /* a pointer violates the alignment rule above                 */
     NVFP4_ERR_MODE = 4,    /* unknown nvfp4_mode                                          */
     NVFP4_ERR_RULE = 5,    /* unknown nvfp4_rule (checked in Four Over Six mode only)     */
-    NVFP4_ERR_CUDA = 6     /* the CUDA runtime reported an error while enqueuing          */
+    NVFP4_ERR_CUDA = 6,    /* the CUDA runtime reported an error while enqueuing          */
+    NVFP4_ERR_VALUE = 7    /* a scalar argument is out of range (nvfp4_qad_kl)            */
 } nvfp4_status;
 
 /* Block-scale selection ([FOS] Problem definition; Core mechanism). */
@@ -156,6 +157,26 @@ NVFP4_API nvfp4_status nvfp4_fakequant(const uint16_t* x, int64_t groups, int64_
 NVFP4_API nvfp4_status nvfp4_quantize_gemm(const uint16_t* x, int64_t rows, int64_t cols, const float* amax,
                                            nvfp4_mode mode, nvfp4_rule rule, uint8_t* codes, uint8_t* scales,
                                            float* tscale, uint8_t* choice, cudaStream_t stream);
+
+/* Distillation loss of quantization-aware distillation ("Quantization-Aware Distillation for
+ * NVFP4 Inference Accuracy Recovery", technical summary §2: the NVFP4 student, whose forward
+ * runs through simulated quantization (nvfp4_fakequant), is trained against the frozen BF16
+ * teacher with L = D_KL(p_teacher || p_student)). For every row r of [rows, vocab] logits:
+ *   p = softmax(teacher[r] / tau), q = softmax(student[r] / tau)
+ *   kl[r]      = sum_v p_v (ln p_v - ln q_v)                    (nats)
+ *   grad[r, v] = BF16(grad_scale * (q_v - p_v))   (d kl[r] / d student[r, v] = (q_v - p_v) / tau:
+ *                pass grad_scale = 1 / (tau * rows) for the gradient of the mean loss)
+ *   teacher, student  [rows, vocab] BF16 bits, 2-byte aligned (16-byte aligned rows with
+ *                     vocab % 8 == 0 take the vectorised path)                     (in)
+ *   kl                [rows] float, 4-byte aligned                                (out)
+ *   grad              NULL, or [rows, vocab] BF16 bits, 2-byte aligned            (out)
+ * Arithmetic in binary32 with an online (single read) softmax per row and the hardware base-2
+ * exponential; the results agree with the binary64 definition to about 1e-6 of the loss's
+ * magnitude (tests/test_gpu_5_qad_kl.py states the bounds). tau must be finite and > 0,
+ * grad_scale finite (else NVFP4_ERR_VALUE); vocab >= 1; logits must be finite. rows == 0 does
+ * nothing. One kernel; a second read of each row when grad is requested. */
+NVFP4_API nvfp4_status nvfp4_qad_kl(const uint16_t* teacher, const uint16_t* student, int64_t rows, int64_t vocab,
+                                    float tau, float grad_scale, float* kl, uint16_t* grad, cudaStream_t stream);
 
 /* Static description of a status code (never NULL). */
 NVFP4_API const char* nvfp4_status_string(nvfp4_status status);

@@ -22,9 +22,10 @@ from typing import NamedTuple
 __all__ = [
     "load", "library_path", "Nvfp4Error",
     "SCALE6", "FOUR_OVER_SIX", "RULE_MAXERR", "RULE_MAE", "RULE_MSE",
-    "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_quantize_gemm",
+    "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_quantize_gemm", "nvfp4_qad_kl",
     "nvfp4_status_string", "nvfp4_version",
     "Quantized", "amax", "quantize", "fakequant", "dequantize", "quantize_for_gemm", "gemm_scale_bytes",
+    "qad_kl", "fakequant_ste",
 ]
 
 SCALE6, FOUR_OVER_SIX = 0, 1
@@ -61,7 +62,9 @@ def load():
         L.nvfp4_dequantize.argtypes = [vp, vp, vp, i64, i64, i64, vp, vp]
         L.nvfp4_fakequant.argtypes = [vp, i64, i64, i64, vp, i32, i32, vp, vp, vp]
         L.nvfp4_quantize_gemm.argtypes = [vp, i64, i64, vp, i32, i32, vp, vp, vp, vp, vp]
-        for f in (L.nvfp4_amax, L.nvfp4_quantize, L.nvfp4_dequantize, L.nvfp4_fakequant, L.nvfp4_quantize_gemm):
+        L.nvfp4_qad_kl.argtypes = [vp, vp, i64, i64, ctypes.c_float, ctypes.c_float, vp, vp, vp]
+        for f in (L.nvfp4_amax, L.nvfp4_quantize, L.nvfp4_dequantize, L.nvfp4_fakequant, L.nvfp4_quantize_gemm,
+                  L.nvfp4_qad_kl):
             f.restype = i32
         L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
         L.nvfp4_version.argtypes, L.nvfp4_version.restype = [], i32
@@ -133,6 +136,11 @@ def nvfp4_quantize_gemm(x, rows, cols, amax, mode, rule, codes, scales, tscale, 
     _check(load().nvfp4_quantize_gemm(_ptr(x), rows, cols, _ptr(amax), _mode(mode), _rule(rule), _ptr(codes),
                                       _ptr(scales), _ptr(tscale), _ptr(choice), _stream(stream)),
            "nvfp4_quantize_gemm")
+
+
+def nvfp4_qad_kl(teacher, student, rows, vocab, tau, grad_scale, kl, grad=None, stream=None):
+    _check(load().nvfp4_qad_kl(_ptr(teacher), _ptr(student), rows, vocab, float(tau), float(grad_scale), _ptr(kl),
+                               _ptr(grad), _stream(stream)), "nvfp4_qad_kl")
 
 
 def nvfp4_status_string(status: int) -> str:
@@ -237,3 +245,38 @@ def quantize_for_gemm(x, mode="four_over_six", rule="mse", amax_values=None, wit
     choice = torch.empty(max(1, (nb + 7) // 8), dtype=torch.uint8, device=dev) if with_choice else None
     nvfp4_quantize_gemm(x, rows, cols, amax_values, mode, rule, codes, scales, tscale, choice, stream)
     return codes, scales, tscale, choice
+
+
+def qad_kl(teacher, student, tau: float = 1.0, grad_scale=None, with_grad: bool = True, stream=None):
+    """Per-row KL(softmax(teacher / tau) || softmax(student / tau)) of [rows, vocab] BF16 logits,
+    and (optionally) grad_scale * (q - p), the gradient of the mean loss when grad_scale is
+    1 / (tau * rows) (the default)."""
+    import torch
+
+    vocab = teacher.shape[-1]
+    rows = teacher.numel() // vocab
+    if student.shape != teacher.shape:
+        raise ValueError("qad_kl: teacher and student shapes differ")
+    if grad_scale is None:
+        grad_scale = 1.0 / (tau * max(rows, 1))
+    kl = torch.empty(rows, dtype=torch.float32, device=teacher.device)
+    grad = torch.empty_like(student, dtype=torch.bfloat16) if with_grad else None
+    nvfp4_qad_kl(teacher, student, rows, vocab, tau, grad_scale, kl, grad, stream)
+    return kl, grad
+
+
+def fakequant_ste(x, mode="four_over_six", rule="mse", groups: int = 1, amax_values=None):
+    """Simulated NVFP4 quantization for a QAD student: the forward is nvfp4_fakequant, the
+    backward passes the gradient through unchanged (straight-through)."""
+    import torch
+
+    class _FakeQuantSTE(torch.autograd.Function):
+        @staticmethod
+        def forward(ctx, inp):
+            return fakequant(inp, mode, rule, groups, amax_values)
+
+        @staticmethod
+        def backward(ctx, g):
+            return g
+
+    return _FakeQuantSTE.apply(x)

@@ -326,6 +326,7 @@ const char* nvfp4_status_string(nvfp4_status status) {
         case NVFP4_ERR_MODE: return "unknown nvfp4_mode";
         case NVFP4_ERR_RULE: return "unknown nvfp4_rule";
         case NVFP4_ERR_CUDA: return "CUDA runtime error while enqueuing work";
+        case NVFP4_ERR_VALUE: return "scalar argument out of range (tau > 0 and finite, grad_scale finite)";
         default: return "unknown nvfp4_status";
     }
 }

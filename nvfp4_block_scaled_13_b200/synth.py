@@ -143,3 +143,20 @@ def random_case(seed: int):
     spread = np.exp2(rng.integers(-20, 21, size=groups)).astype(np.float32)
     x = (x.reshape(groups, -1) * spread[:, None]).ravel()
     return to_bf16_bits(x), (groups, rows, cols)
+
+
+def qad_logits(rows: int, vocab: int, seed: int = 5, noise: float = 0.3, scale: float = 3.0, peaked: float = 0.25):
+    """Teacher and student logits for the QAD loss, as BF16 bits [rows, vocab].
+
+    Stand-in for a frozen teacher and an NVFP4 student on the same tokens (no model or data
+    is available): teacher logits N(0, scale^2) with a fraction `peaked` of rows made
+    confident (one logit raised by 4 * scale); the student is the teacher plus N(0, noise^2),
+    the small disagreement that quantization noise leaves."""
+    rng = np.random.default_rng(seed)
+    t = rng.standard_normal((rows, vocab), dtype=np.float32) * np.float32(scale)
+    npk = int(rows * peaked)
+    if npk and vocab > 1:
+        idx = rng.integers(0, vocab, npk)
+        t[np.arange(npk), idx] += np.float32(4 * scale)
+    s = t + rng.standard_normal((rows, vocab), dtype=np.float32) * np.float32(noise)
+    return to_bf16_bits(t).reshape(rows, vocab), to_bf16_bits(s).reshape(rows, vocab)

@@ -19,7 +19,7 @@ def header_functions(path):
 
 def test_header_declares_the_boundary():
     names = header_functions(os.path.join(ROOT, "include", "nvfp4.h"))
-    assert names == ["nvfp4_amax", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_quantize",
+    assert names == ["nvfp4_amax", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_qad_kl", "nvfp4_quantize",
                      "nvfp4_quantize_gemm", "nvfp4_status_string", "nvfp4_version"]
 
 
@@ -32,7 +32,7 @@ def test_library_exports_every_declared_symbol():
 def test_status_strings_and_version():
     assert nv.nvfp4_version() == 100
     assert nv.nvfp4_status_string(0) == "ok"
-    for s in range(1, 7):
+    for s in range(1, 8):
         assert nv.nvfp4_status_string(s) not in ("ok", "unknown nvfp4_status")
     assert nv.nvfp4_status_string(99) == "unknown nvfp4_status"
 
@@ -76,6 +76,16 @@ A = 1 << 20          # 32-byte aligned
     (lambda L: L.nvfp4_quantize_gemm(A, 4, 32, A, 3, 2, A, A, A, None, None), 4),
     (lambda L: L.nvfp4_quantize_gemm(A, 4, 32, A, 1, 7, A, A, A, None, None), 5),
     (lambda L: L.nvfp4_quantize_gemm(A + 8, 4, 32, A, 1, 2, A, A, A, None, None), 3),
+    # nvfp4_qad_kl(teacher, student, rows, vocab, tau, grad_scale, kl, grad, stream)
+    (lambda L: L.nvfp4_qad_kl(A, A, 4, 0, 1.0, 1.0, A, None, None), 2),
+    (lambda L: L.nvfp4_qad_kl(A, A, -1, 8, 1.0, 1.0, A, None, None), 2),
+    (lambda L: L.nvfp4_qad_kl(A, A, 4, 8, 0.0, 1.0, A, None, None), 7),
+    (lambda L: L.nvfp4_qad_kl(A, A, 4, 8, float("inf"), 1.0, A, None, None), 7),
+    (lambda L: L.nvfp4_qad_kl(A, A, 4, 8, 1.0, float("nan"), A, None, None), 7),
+    (lambda L: L.nvfp4_qad_kl(None, A, 4, 8, 1.0, 1.0, A, None, None), 1),
+    (lambda L: L.nvfp4_qad_kl(A, A, 4, 8, 1.0, 1.0, None, None, None), 1),
+    (lambda L: L.nvfp4_qad_kl(A + 1, A, 4, 8, 1.0, 1.0, A, None, None), 3),
+    (lambda L: L.nvfp4_qad_kl(A, A, 4, 8, 1.0, 1.0, A + 2, None, None), 3),
     # nvfp4_fakequant(x, G, R, C, amax, mode, rule, y, choice, stream)
     (lambda L: L.nvfp4_fakequant(A, 1, 4, 32, A, 1, 2, None, None, None), 1),
     (lambda L: L.nvfp4_fakequant(A, 1, 4, 32, A, 7, 2, A, None, None), 4),
