@@ -87,11 +87,12 @@ __device__ __forceinline__ float recip_clamped(float d) {
     return d > 0.0f ? fminf(__frcp_rn(d), FLT_MAX) : 0.0f;
 }
 
-// Per-group constants: alpha = amax / (6 M), beta_K = K * alpha, and the reciprocals of the
-// betas used to bracket the block-scale quotients (valid when both lie in [2^-125, 2^125],
-// so that the reciprocals are normal numbers within half an ulp).
+// Per-group constants: alpha = amax / (6 M), beta_K = K * alpha, and the bracket factors
+// yl_K = RN(RN(1/beta_K) * (1 - 2^-20)), yh_K = RN(RN(1/beta_K) * (1 + 2^-20)) used to bracket
+// the block-scale quotients (valid when both betas lie in [2^-125, 2^125], so that every
+// factor is a normal number).
 struct GroupCtx {
-    float alpha, beta6, beta4, y6, y4;
+    float alpha, beta6, beta4, yl6, yh6, yl4, yh4;
     bool fast;
 };
 
@@ -103,28 +104,33 @@ __device__ __forceinline__ GroupCtx make_group(float amax, float six_m) {
     c.beta4 = __fmul_rn(4.0f, c.alpha);
     const float lo = FOUR ? c.beta4 : c.beta6;
     c.fast = lo >= 0x1p-125f && c.beta6 <= 0x1p125f;
-    c.y6 = c.fast ? __frcp_rn(c.beta6) : 0.0f;
-    c.y4 = c.fast ? __frcp_rn(c.beta4) : 0.0f;
+    constexpr float kLo = 1.0f - 0x1p-20f, kHi = 1.0f + 0x1p-20f;
+    const float y6 = c.fast ? __frcp_rn(c.beta6) : 0.0f, y4 = c.fast ? __frcp_rn(c.beta4) : 0.0f;
+    c.yl6 = __fmul_rn(y6, kLo);
+    c.yh6 = __fmul_rn(y6, kHi);
+    c.yl4 = __fmul_rn(y4, kLo);
+    c.yh4 = __fmul_rn(y4, kHi);
     return c;
 }
 
 // E4M3(RN(m / beta_6)) in the low byte and E4M3(RN(m / beta_4)) in the high byte.
-// t' = RN(m * RN(1/beta)) is within 3 ulps of RN(m / beta); scaling it by 1 -+ 2^-20 gives a
-// bracket that contains RN(m / beta), and E4M3 rounding is monotone, so equal conversions of
-// the two ends are the exact scale. Near a boundary, or outside the bracket's valid range,
-// the exact division decides.
+// lo = RN(m * yl) and hi = RN(m * yh) carry three roundings of at most 2^-24 each on top of
+// the factors 1 -+ 2^-20, so lo < m/beta * (1 - 2^-21) < RN(m / beta) < hi whenever the
+// products are normal; below 2^-126 every one of them converts to E4M3 zero, and an overflow
+// saturates to 448 like the quotient it bounds. E4M3 rounding is monotone, so equal
+// conversions of lo and hi are the exact scale. Near a rounding boundary (about one block in
+// 2^15), or outside the factors' valid range, the exact division decides.
 template <bool FOUR>
 __device__ __forceinline__ uint32_t block_scales(float m, const GroupCtx& c) {
     if (c.fast) {
-        constexpr float kLo = 1.0f - 0x1p-20f, kHi = 1.0f + 0x1p-20f;
         if (FOUR) {
-            const float2 t = mul2(make_float2(m, m), make_float2(c.y6, c.y4));
-            const float2 lo = mul2(t, make_float2(kLo, kLo)), hi = mul2(t, make_float2(kHi, kHi));
-            const uint32_t w = e4m3x2(lo.x, hi.x) | (e4m3x2(lo.y, hi.y) << 16);   // lo6 hi6 lo4 hi4
-            if (((w ^ (w >> 8)) & 0x00FF00FFu) == 0u) return __byte_perm(w, 0u, 0x4420);
+            const float2 lo = mul2(make_float2(m, m), make_float2(c.yl6, c.yl4));
+            const float2 hi = mul2(make_float2(m, m), make_float2(c.yh6, c.yh4));
+            const uint32_t wl = e4m3x2(lo.x, lo.y), wh = e4m3x2(hi.x, hi.y);
+            if (wl == wh) return wl;
         } else {
-            const float t6 = __fmul_rn(m, c.y6);
-            const uint32_t b6 = e4m3x2(__fmul_rn(t6, kLo), __fmul_rn(t6, kHi));
+            const float2 b = mul2(make_float2(m, m), make_float2(c.yl6, c.yh6));
+            const uint32_t b6 = e4m3x2(b.x, b.y);
             if ((b6 & 0xFFu) == (b6 >> 8)) return b6 & 0xFFu;
         }
     }
@@ -170,33 +176,39 @@ __device__ __forceinline__ float candidate(const float2 (&x)[8], float r, float 
 }
 
 // Quantize the block in `w` (eight BF16 pairs). Stores its codes + scale (or fake-quant
-// BF16) and returns whether target 4 was kept. TABLE: d and 1/d come from `tab`.
+// BF16) and returns whether target 4 was kept. TABLE: d and 1/d come from `tab`. ok = false
+// (a lane past the end of the group) computes but stores nothing and returns false.
 template <bool FOUR, int RULE, bool FQ, bool TABLE>
 __device__ __forceinline__ bool quantize_block(const uint32_t (&w)[8], const GroupCtx& gc, const float2* tab,
-                                               uint8_t* codes8, uint8_t* scale1, uint16_t* y16) {
+                                               uint8_t* codes8, uint8_t* scale1, uint16_t* y16, bool ok = true) {
     float2 x[8];
-    float m = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        x[j] = unpack_bf16x2(w[j]);
-        m = max3(m, fabsf(x[j].x), fabsf(x[j].y));
-    }
+    for (int j = 0; j < 8; ++j) x[j] = unpack_bf16x2(w[j]);
+    // max over {0, |x_i|}: depth-3 tree of 3-input max (the same value as a running max)
+    const float m01 = max3(0.0f, fabsf(x[0].x), fabsf(x[0].y));
+    const float m02 = max3(fabsf(x[1].x), fabsf(x[1].y), fabsf(x[2].x));
+    const float m03 = max3(fabsf(x[2].y), fabsf(x[3].x), fabsf(x[3].y));
+    const float m04 = max3(fabsf(x[4].x), fabsf(x[4].y), fabsf(x[5].x));
+    const float m05 = max3(fabsf(x[5].y), fabsf(x[6].x), fabsf(x[6].y));
+    const float m06 = max3(fabsf(x[7].x), fabsf(x[7].y), 0.0f);
+    const float m = fmaxf(max3(m01, m02, m03), max3(m04, m05, m06));
     const uint32_t s2 = block_scales<FOUR>(m, gc);
-    const float2 e6 = TABLE ? tab[s2 & 0xFFu] : scale_entry(s2 & 0xFFu, gc.alpha);
+    const uint32_t i6 = __byte_perm(s2, 0u, 0x4440), i4 = __byte_perm(s2, 0u, 0x4441);
+    const float2 e6 = TABLE ? tab[i6] : scale_entry(i6, gc.alpha);
     uint32_t clo, chi, h[8];
     const float err6 = candidate<RULE>(x, e6.y, e6.x, clo, chi, h);
-    uint32_t s = s2 & 0xFFu;
+    uint32_t s = i6;
     float dsel = e6.x;
     bool four = false;
     if (FOUR) {
-        const float2 e4 = TABLE ? tab[s2 >> 8] : scale_entry(s2 >> 8, gc.alpha);
+        const float2 e4 = TABLE ? tab[i4] : scale_entry(i4, gc.alpha);
         uint32_t c4lo, c4hi, h4[8];
         const float err4 = candidate<RULE>(x, e4.y, e4.x, c4lo, c4hi, h4);
         four = err4 < err6;   // ties keep target 6
         if (four) {
             clo = c4lo;
             chi = c4hi;
-            s = s2 >> 8;
+            s = i4;
             dsel = e4.x;
         }
         if (FQ) {
@@ -209,12 +221,12 @@ __device__ __forceinline__ bool quantize_block(const uint32_t (&w)[8], const Gro
         uint32_t out[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) out[j] = bf16x2(mul2(f16x2_to_float2(h[j]), dd));
-        st32(y16, out);
-    } else {
+        if (ok) st32(y16, out);
+    } else if (ok) {
         st8(codes8, clo, chi);
         *scale1 = static_cast<uint8_t>(s);
     }
-    return four;
+    return four && ok;
 }
 
 // Byte offset of local block a's scale in the tiled layout: 128-row x 4-column tiles of 512
@@ -291,11 +303,49 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
 // Grid: x = CTAs per group, y = groups (looping when there are more than gridDim.y).
 // Each warp works on tiles of 64 consecutive blocks of its group: lane t quantizes blocks t and
 // t + 32 of the tile, so both 32-byte loads, both code stores and both scale stores of a warp
-// are contiguous, and each half-tile's 32 choice bits are one ballot word. The next tile's two
-// blocks are loaded before the current ones are worked on.
+// are contiguous, and each half-tile's 32 choice bits are one ballot word. The next tile's
+// blocks are loaded into registers before the current ones are worked on: in 4/6 mode into a
+// second register set (the loop is unrolled twice so the two sets swap roles without copies),
+// in scale-6 mode into one set that is copied, which keeps that kernel within 64 registers.
+// The last, partial tile runs the same code with its stores predicated off.
 // Requires every group to start on a 32-block boundary of the flat index (one group, or
 // blocks_per_group % 32 == 0) and blocks_per_group < 2^30.
 // SWZ: scales go to the tiled GEMM layout (one group only).
+// One warp tile (64 blocks) of one group; lane t works on blocks 64 tile + t and + 32.
+template <bool FOUR, int RULE, bool FQ, bool SWZ>
+__device__ __forceinline__ void quant_tile(const QuantParams& p, const GroupCtx& gc, const float2* tab,
+                                           uint32_t tile, uint32_t lane, uint32_t bpg, uint8_t* cg, uint8_t* sg,
+                                           uint16_t* yg, uint32_t* chw, int64_t chw_left, int64_t base,
+                                           const uint32_t (&ca)[8], const uint32_t (&cb)[8]) {
+    const uint32_t a = (tile << 6) + lane;
+    const bool oka = a < bpg, okb = a + 32u < bpg;
+    const bool fa = quantize_block<FOUR, RULE, FQ, true>(ca, gc, tab, FQ ? nullptr : cg + static_cast<size_t>(a) * 8,
+                                                         FQ ? nullptr : (SWZ ? p.scales + tiled_scale_offset(a, p) : sg + a),
+                                                         FQ ? yg + static_cast<size_t>(a) * 16 : nullptr, oka);
+    const bool fb = quantize_block<FOUR, RULE, FQ, true>(cb, gc, tab, FQ ? nullptr : cg + static_cast<size_t>(a + 32u) * 8,
+                                                         FQ ? nullptr : (SWZ ? p.scales + tiled_scale_offset(a + 32u, p) : sg + a + 32u),
+                                                         FQ ? yg + static_cast<size_t>(a + 32u) * 16 : nullptr, okb);
+    if (p.choice != nullptr) {
+        const uint32_t bits_a = __ballot_sync(0xFFFFFFFFu, fa);
+        const uint32_t bits_b = __ballot_sync(0xFFFFFFFFu, fb);
+        const uint32_t w = 2u * tile + lane;
+        if (lane < 2u && (w << 5) < bpg) {
+            const uint32_t bits = lane ? bits_b : bits_a;
+            if (static_cast<int64_t>(w) < chw_left) chw[w] = bits;
+            else store_choice(p.choice, p.choice_bytes, base + (static_cast<int64_t>(w) << 5), bits);
+        }
+    }
+}
+
+// Load a lane's two blocks of a tile. Lanes past the group's end (bpg >= 1) re-read its last
+// block, so every register the tile computes on holds defined data; their stores are off.
+__device__ __forceinline__ void load_tile(const uint16_t* xg, uint32_t tile, uint32_t lane, uint32_t bpg,
+                                          uint32_t (&ra)[8], uint32_t (&rb)[8]) {
+    const uint32_t a = (tile << 6) + lane, last = bpg - 1u;
+    ld32_stream(xg + static_cast<size_t>(min(a, last)) * 16, ra);
+    ld32_stream(xg + static_cast<size_t>(min(a + 32u, last)) * 16, rb);
+}
+
 template <bool FOUR, int RULE, bool FQ, bool SWZ = false>
 __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kernel(const QuantParams p) {
     constexpr float kSixM = FOUR ? 1536.0f : 2688.0f;   // 6 * 256 or 6 * 448
@@ -320,54 +370,31 @@ __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kerne
         uint32_t* chw = reinterpret_cast<uint32_t*>(p.choice) + (base >> 5);   // base is a multiple of 32
         const int64_t chw_left = choice_words - (base >> 5);
         uint32_t tile = warp0;
-        uint32_t na[8], nb[8];
-        {
-            const uint32_t a = (tile << 6) + lane;
-            if (tile < ntiles && a < bpg) ld32_stream(xg + static_cast<size_t>(a) * 16, na);
-            if (tile < ntiles && a + 32u < bpg) ld32_stream(xg + static_cast<size_t>(a + 32u) * 16, nb);
-        }
-        for (; tile < ntiles; tile += warps) {
-            uint32_t ca[8], cb[8];
+        uint32_t a0[8], a1[8];
+        if (tile < ntiles) load_tile(xg, tile, lane, bpg, a0, a1);
+        if constexpr (!FOUR) {   // one prefetch buffer: two would not fit the 64-register budget
+            for (; tile < ntiles; tile += warps) {
+                uint32_t b0[8], b1[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                ca[k] = na[k];
-                cb[k] = nb[k];
-            }
-            const uint32_t a = (tile << 6) + lane;
-            const uint32_t an = ((tile + warps) << 6) + lane;
-            if (tile + warps < ntiles) {
-                if (an < bpg) ld32_stream(xg + static_cast<size_t>(an) * 16, na);
-                if (an + 32u < bpg) ld32_stream(xg + static_cast<size_t>(an + 32u) * 16, nb);
-            }
-            bool fa = false, fb = false;
-            if ((tile << 6) + 64u <= bpg) {    // interior tile: all 64 blocks exist (warp-uniform)
-                fa = quantize_block<FOUR, RULE, FQ, true>(ca, gc, tab, FQ ? nullptr : cg + static_cast<size_t>(a) * 8,
-                                                          FQ ? nullptr : (SWZ ? p.scales + tiled_scale_offset(a, p) : sg + a),
-                                                          FQ ? yg + static_cast<size_t>(a) * 16 : nullptr);
-                fb = quantize_block<FOUR, RULE, FQ, true>(cb, gc, tab, FQ ? nullptr : cg + static_cast<size_t>(a + 32u) * 8,
-                                                          FQ ? nullptr : (SWZ ? p.scales + tiled_scale_offset(a + 32u, p) : sg + a + 32u),
-                                                          FQ ? yg + static_cast<size_t>(a + 32u) * 16 : nullptr);
-            } else {
-                if (a < bpg)
-                    fa = quantize_block<FOUR, RULE, FQ, true>(ca, gc, tab, FQ ? nullptr : cg + static_cast<size_t>(a) * 8,
-                                                              FQ ? nullptr : (SWZ ? p.scales + tiled_scale_offset(a, p) : sg + a),
-                                                              FQ ? yg + static_cast<size_t>(a) * 16 : nullptr);
-                if (a + 32u < bpg)
-                    fb = quantize_block<FOUR, RULE, FQ, true>(cb, gc, tab,
-                                                              FQ ? nullptr : cg + static_cast<size_t>(a + 32u) * 8,
-                                                              FQ ? nullptr : (SWZ ? p.scales + tiled_scale_offset(a + 32u, p) : sg + a + 32u),
-                                                              FQ ? yg + static_cast<size_t>(a + 32u) * 16 : nullptr);
-            }
-            if (p.choice != nullptr) {
-                const uint32_t bits_a = __ballot_sync(0xFFFFFFFFu, fa);
-                const uint32_t bits_b = __ballot_sync(0xFFFFFFFFu, fb);
-                // lane 0 stores the word of blocks [64 tile, +32), lane 1 the next one (if any)
-                const uint32_t w = 2u * tile + lane;
-                if (lane < 2u && (w << 5) < bpg) {
-                    const uint32_t bits = lane ? bits_b : bits_a;
-                    if (static_cast<int64_t>(w) < chw_left) chw[w] = bits;
-                    else store_choice(p.choice, p.choice_bytes, base + (static_cast<int64_t>(w) << 5), bits);
+                for (int k = 0; k < 8; ++k) {
+                    b0[k] = a0[k];
+                    b1[k] = a1[k];
                 }
+                if (tile + warps < ntiles) load_tile(xg, tile + warps, lane, bpg, a0, a1);
+                quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, chw_left, base, b0, b1);
+            }
+        } else {
+            uint32_t b0[8], b1[8];
+            while (tile < ntiles) {
+                uint32_t nt = tile + warps;
+                if (nt < ntiles) load_tile(xg, nt, lane, bpg, b0, b1);
+                quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, chw_left, base, a0, a1);
+                tile = nt;
+                if (tile >= ntiles) break;
+                nt = tile + warps;
+                if (nt < ntiles) load_tile(xg, nt, lane, bpg, a0, a1);
+                quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, chw_left, base, b0, b1);
+                tile = nt;
             }
         }
     }
