@@ -315,23 +315,26 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
 template <bool FOUR, int RULE, bool FQ, bool SWZ>
 __device__ __forceinline__ void quant_tile(const QuantParams& p, const GroupCtx& gc, const float2* tab,
                                            uint32_t tile, uint32_t lane, uint32_t bpg, uint8_t* cg, uint8_t* sg,
-                                           uint16_t* yg, uint32_t* chw, int64_t chw_left, int64_t base,
+                                           uint16_t* yg, uint32_t* chw, int64_t base,
                                            const uint32_t (&ca)[8], const uint32_t (&cb)[8]) {
     const uint32_t a = (tile << 6) + lane;
     const bool oka = a < bpg, okb = a + 32u < bpg;
-    const bool fa = quantize_block<FOUR, RULE, FQ, true>(ca, gc, tab, FQ ? nullptr : cg + static_cast<size_t>(a) * 8,
-                                                         FQ ? nullptr : (SWZ ? p.scales + tiled_scale_offset(a, p) : sg + a),
-                                                         FQ ? yg + static_cast<size_t>(a) * 16 : nullptr, oka);
-    const bool fb = quantize_block<FOUR, RULE, FQ, true>(cb, gc, tab, FQ ? nullptr : cg + static_cast<size_t>(a + 32u) * 8,
-                                                         FQ ? nullptr : (SWZ ? p.scales + tiled_scale_offset(a + 32u, p) : sg + a + 32u),
-                                                         FQ ? yg + static_cast<size_t>(a + 32u) * 16 : nullptr, okb);
+    // the second block's addresses are the first one's plus constant offsets (32 blocks)
+    uint8_t* c0 = FQ ? nullptr : cg + static_cast<size_t>(a) * 8;
+    uint8_t* s0 = FQ ? nullptr : sg + a;
+    uint16_t* y0 = FQ ? yg + static_cast<size_t>(a) * 16 : nullptr;
+    const bool fa = quantize_block<FOUR, RULE, FQ, true>(ca, gc, tab, c0, SWZ ? p.scales + tiled_scale_offset(a, p) : s0,
+                                                         y0, oka);
+    const bool fb = quantize_block<FOUR, RULE, FQ, true>(cb, gc, tab, FQ ? nullptr : c0 + 256,
+                                                         SWZ ? p.scales + tiled_scale_offset(a + 32u, p) : (FQ ? nullptr : s0 + 32),
+                                                         FQ ? y0 + 512 : nullptr, okb);
     if (p.choice != nullptr) {
         const uint32_t bits_a = __ballot_sync(0xFFFFFFFFu, fa);
         const uint32_t bits_b = __ballot_sync(0xFFFFFFFFu, fb);
         const uint32_t w = 2u * tile + lane;
         if (lane < 2u && (w << 5) < bpg) {
             const uint32_t bits = lane ? bits_b : bits_a;
-            if (static_cast<int64_t>(w) < chw_left) chw[w] = bits;
+            if ((w << 5) + 32u <= bpg) chw[w] = bits;   // all 32 blocks of the word exist
             else store_choice(p.choice, p.choice_bytes, base + (static_cast<int64_t>(w) << 5), bits);
         }
     }
@@ -355,7 +358,6 @@ __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kerne
     const uint32_t ntiles = (bpg + 63u) >> 6;
     const uint32_t warps = gridDim.x * (kThreads / 32);
     const uint32_t warp0 = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
-    const int64_t choice_words = p.choice_bytes >> 2;          // whole 32-bit words of the bitmap
     for (int64_t g = blockIdx.y; g < p.groups; g += gridDim.y) {
         const GroupCtx gc = make_group<FOUR>(__ldg(p.amax + g), kSixM);
         __syncthreads();                       // the previous group's table is no longer read
@@ -368,7 +370,6 @@ __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kerne
         uint8_t* sg = FQ ? nullptr : p.scales + base;
         uint16_t* yg = FQ ? p.y + base * 16 : nullptr;
         uint32_t* chw = reinterpret_cast<uint32_t*>(p.choice) + (base >> 5);   // base is a multiple of 32
-        const int64_t chw_left = choice_words - (base >> 5);
         uint32_t tile = warp0;
         uint32_t a0[8], a1[8];
         if (tile < ntiles) load_tile(xg, tile, lane, bpg, a0, a1);
@@ -381,19 +382,19 @@ __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kerne
                     b1[k] = a1[k];
                 }
                 if (tile + warps < ntiles) load_tile(xg, tile + warps, lane, bpg, a0, a1);
-                quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, chw_left, base, b0, b1);
+                quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, base, b0, b1);
             }
         } else {
             uint32_t b0[8], b1[8];
             while (tile < ntiles) {
                 uint32_t nt = tile + warps;
                 if (nt < ntiles) load_tile(xg, nt, lane, bpg, b0, b1);
-                quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, chw_left, base, a0, a1);
+                quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, base, a0, a1);
                 tile = nt;
                 if (tile >= ntiles) break;
                 nt = tile + warps;
                 if (nt < ntiles) load_tile(xg, nt, lane, bpg, a0, a1);
-                quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, chw_left, base, b0, b1);
+                quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, base, b0, b1);
                 tile = nt;
             }
         }
