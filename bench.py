@@ -43,6 +43,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle leg")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-per-config", action="store_true", help="skip the per-workload leg")
     ap.add_argument("--rows", type=int, default=None,
                     help="rows of the 65536 x 8192 workload to use (default: all; smaller slices for tests)")
     return ap.parse_args()
@@ -201,24 +202,56 @@ def make_input(rank: int, rows=None):
 
 # ---- CPU oracle legs -----------------------------------------------------------------------
 
-def oracle_step(x_rows: np.ndarray, rows: int, cols: int):
+def host_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def oracle_step(x_rows: np.ndarray, rows: int, cols: int, threads: int = 1):
+    """amax, quantize (amax given) and dequantize by the oracle, its C functions called on
+    `threads` row ranges at once (the oracle's calls release the interpreter lock and blocks
+    are independent, so the ranges give the same bytes as one call over all rows)."""
     import oracle as O
 
-    a = O.amax(x_rows, 1, rows, cols)
-    q = O.quantize(x_rows, 1, rows, cols, a, MODE, RULE)
-    O.dequantize(q["codes"], q["scales"], q["tscale"], 1, rows, cols)
+    O.lib()
+    if threads <= 1:
+        a = O.amax(x_rows, 1, rows, cols)
+        q = O.quantize(x_rows, 1, rows, cols, a, MODE, RULE)
+        O.dequantize(q["codes"], q["scales"], q["tscale"], 1, rows, cols)
+        return
+    from concurrent.futures import ThreadPoolExecutor
+
+    bounds = [(rows * i // threads, rows * (i + 1) // threads) for i in range(threads)]
+    bounds = [(lo, hi) for lo, hi in bounds if hi > lo]
+    part = lambda lo, hi: x_rows[lo * cols:hi * cols]
+    with ThreadPoolExecutor(len(bounds)) as ex:
+        a = np.max(list(ex.map(lambda b: O.amax(part(*b), 1, b[1] - b[0], cols), bounds)), axis=0)
+
+        def rest(b):
+            q = O.quantize(part(*b), 1, b[1] - b[0], cols, a, MODE, RULE)
+            O.dequantize(q["codes"], q["scales"], q["tscale"], 1, b[1] - b[0], cols)
+
+        list(ex.map(rest, bounds))
 
 
 def cpu_baseline(x: np.ndarray, cols: int, rows: int = 12288):
-    """The oracle as it stands (C, one thread) on the first `rows` rows of the workload."""
+    """The oracle as it stands (C) on the first `rows` rows of the workload: on all host
+    cores (the reported value), and on one thread."""
     xs = np.ascontiguousarray(x[: rows * cols])
+    threads = host_threads()
     t0 = time.perf_counter()
-    oracle_step(xs, rows, cols)
-    dt = time.perf_counter() - t0
-    return {"value": round(2 * rows * cols / dt / GB, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+    oracle_step(xs, rows, cols, threads)
+    dt_all = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle_step(xs, rows, cols, 1)
+    dt_one = time.perf_counter() - t0
+    return {"value": round(2 * rows * cols / dt_all / GB, 5), "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": f"rows 0..{rows - 1} of the 65536x8192 tensor ({rows * cols / 1e6:.1f} M elements): "
-                      f"amax + 4/6-MSE quantize + dequantize, single thread, {dt:.1f} s",
-            "seconds": round(dt, 2)}
+                      f"amax + 4/6-MSE quantize + dequantize on {threads} threads ({dt_all:.2f} s); "
+                      f"one thread: {dt_one:.1f} s",
+            "single_thread": {"value": round(2 * rows * cols / dt_one / GB, 5), "unit": "GB/s"}}
 
 
 def run_reference(args, rank, world):
@@ -226,22 +259,24 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     x, (g, r, c) = make_input(0, args.rows)
+    threads = host_threads()
     # calibrate, then size each step's sample so that the whole run takes about two minutes
-    cal_rows = 64
+    cal_rows = 16 * threads
     t0 = time.perf_counter()
-    oracle_step(np.ascontiguousarray(x[: cal_rows * c]), cal_rows, c)
+    oracle_step(np.ascontiguousarray(x[: cal_rows * c]), cal_rows, c, threads)
     per_row = (time.perf_counter() - t0) / cal_rows
-    rows = int(max(1, min(4096, r // 2, 120.0 / max(1, args.steps + args.warmup) / per_row)))
+    rows = int(max(threads, min(8192, r // 2, 120.0 / max(1, args.steps + args.warmup) / per_row)))
     for i in range(args.warmup):
         s = (i * rows) % (r - rows)
-        oracle_step(np.ascontiguousarray(x[s * c:(s + rows) * c]), rows, c)
+        oracle_step(np.ascontiguousarray(x[s * c:(s + rows) * c]), rows, c, threads)
     t0 = time.perf_counter()
     for i in range(args.steps):
         s = ((args.warmup + i) * rows) % (r - rows)
-        oracle_step(np.ascontiguousarray(x[s * c:(s + rows) * c]), rows, c)
+        oracle_step(np.ascontiguousarray(x[s * c:(s + rows) * c]), rows, c, threads)
     dt = time.perf_counter() - t0
     value = 2 * rows * c * args.steps / dt / GB
-    sample = f"{rows} rows x 8192 per step ({rows * c / 1e6:.2f} M elements): amax + 4/6-MSE quantize + dequantize"
+    sample = (f"{rows} rows x 8192 per step ({rows * c / 1e6:.2f} M elements): amax + 4/6-MSE quantize + "
+              f"dequantize on {threads} threads")
     print(json.dumps({
         "impl": "reference", "metric": "NVFP4 quantize input GB/s & % of B200 HBM peak; 4/6 overhead vs scale-6",
         "value": round(value, 6), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -249,12 +284,145 @@ def run_reference(args, rank, world):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": f"c5: BF16 {r}x{c} N(0,1), 1% zero blocks, 1% blocks x1e-6; "
                                "Four Over Six, MSE rule", "shape": [1, r, c], "step": "amax + quantize + dequantize"},
-        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
 
 # ---- GPU legs ------------------------------------------------------------------------------
+
+L2_BYTES = 126 * 2**20
+
+
+def per_config_leg(nv, torch, dev, stream, peak, resident=None):
+    """The quantize kernel on each workload with its amax given (the fixed-scale path): time,
+    input GB/s (2N / t), algorithmic bytes / t against the HBM peak, amax + quantize, and the
+    Four Over Six overhead against scale-6 timed in interleaved repetitions on the same tensor.
+    Inputs that fit in L2 are timed cold (a 512 MiB write flushes L2 before each launch) and
+    warm (back to back); the 512 KiB workload is timed by CUDA-graph replay of 50 launches."""
+    from nvfp4_block_scaled_13_b200 import synth
+
+    s = stream.cuda_stream
+    flush = torch.empty(512 * 2**20, dtype=torch.uint8, device=dev)
+    modes = {"scale6": 0, "four_over_six": 1}
+    rules = {"maxerr": 0, "mae": 1, "mse": 2}
+    out = {}
+    for name, cfg in synth.CONFIGS.items():
+        x, (g, r, c) = resident[name] if resident and name in resident else synth.make(name)
+        n, nb = g * r * c, g * r * c // 16
+        xd = torch.from_numpy(x.view(np.int16)).to(dev)
+        del x
+        amax = torch.empty(g, dtype=torch.float32, device=dev)
+        tscale = torch.empty(g, dtype=torch.float32, device=dev)
+        choice = torch.empty((nb + 7) // 8, dtype=torch.uint8, device=dev)
+        fq = cfg.output == "fakequant"
+        if fq:
+            y = torch.empty(n, dtype=torch.int16, device=dev)
+            nbytes = 4 * n + (nb + 7) // 8 + 4 * g
+        else:
+            codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+            scales = torch.empty(nb, dtype=torch.uint8, device=dev)
+            nbytes = algorithmic_bytes(n, g)["quantize"]
+
+        def launch(mode, rule):   # on the current stream (a graph's capture stream while capturing)
+            cs = torch.cuda.current_stream(dev).cuda_stream
+            if fq:
+                nv.nvfp4_fakequant(xd, g, r, c, amax, mode, rule, y, choice, cs)
+            else:
+                nv.nvfp4_quantize(xd, g, r, c, amax, mode, rule, codes, scales, tscale, choice, cs)
+
+        nv.nvfp4_amax(xd, g, r, c, amax, s)
+        variants = [("scale6", 0, 2)]
+        if cfg.mode == "four_over_six":
+            names = ["maxerr", "mae", "mse"] if name == WORKLOAD else [cfg.rule]
+            variants += [(f"46_{k}", 1, rules[k]) for k in names]
+        for v in variants:
+            launch(v[1], v[2])
+        torch.cuda.synchronize(dev)
+        small = 2 * n <= 4 * 2**20
+        fits_l2 = 2 * n <= L2_BYTES
+        res = {"shape": [g, r, c], "output": cfg.output, "bytes_per_launch": nbytes}
+
+        def timed(fn, cold):
+            if cold:
+                flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            return a.elapsed_time(b)
+
+        if small:
+            per = {}
+            for vname, mode, rule in variants:
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph):
+                    for _ in range(50):
+                        launch(mode, rule)
+                graph.replay()
+                torch.cuda.synchronize(dev)
+                reps = []
+                for _ in range(10):
+                    reps.append(timed(graph.replay, False) / 50)
+                per[vname] = statistics.median(reps)
+                del graph
+            res["timing"] = "warm, CUDA-graph replay of 50 launches"
+        else:
+            kinds = [("cold", True), ("warm", False)] if fits_l2 else [("", False)]
+            per = {}
+            for kind, cold in kinds:
+                t = {v[0]: [] for v in variants}
+                for rep_i in range(14):
+                    for vname, mode, rule in (variants if rep_i % 2 == 0 else variants[::-1]):
+                        dt = timed(lambda: launch(mode, rule), cold)
+                        if rep_i >= 2:
+                            t[vname].append(dt)
+                for vname in t:
+                    per[vname + (f"_{kind}" if kind else "")] = statistics.median(t[vname])
+            res["timing"] = ("L2 flushed before each launch (cold) and back to back (warm)" if fits_l2
+                             else "back to back; the input is larger than L2")
+        main_v = variants[-1][0]
+        suffix = "_cold" if (fits_l2 and not small) else ""
+        tq = per[main_v + suffix]
+        res["ms"] = {k: round(v, 5) for k, v in per.items()}
+        res["kernel"] = f"{'fakequant' if fq else 'quantize'} {main_v}"
+        res["input_GBps"] = round(2 * n / (tq * 1e-3) / GB, 1)
+        res["GBps"] = round(nbytes / (tq * 1e-3) / GB, 1)
+        res["frac_of_peak"] = round(nbytes / (tq * 1e-3) / GB / peak, 4)
+        if len(variants) > 1:
+            res["overhead_46_vs_scale6"] = {
+                k[3:]: round(per[k + suffix] / per["scale6" + suffix] - 1.0, 4) for k, _, _ in variants[1:]}
+        def both():
+            nv.nvfp4_amax(xd, g, r, c, amax, torch.cuda.current_stream(dev).cuda_stream)
+            launch(variants[-1][1], variants[-1][2])
+
+        t_aq = []
+        if small:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for _ in range(50):
+                    both()
+            graph.replay()
+            torch.cuda.synchronize(dev)
+            t_aq = [timed(graph.replay, False) / 50 for _ in range(10)]
+            del graph
+        else:
+            for rep_i in range(8):
+                dt = timed(both, fits_l2)
+                if rep_i >= 2:
+                    t_aq.append(dt)
+        res["amax_plus_quantize_ms"] = round(statistics.median(t_aq), 5)
+        out[name] = res
+        del xd
+        if fq:
+            del y
+        else:
+            del codes, scales
+    del flush
+    torch.cuda.empty_cache()
+    return out
 
 def run_ours(args, rank, world, local):
     import torch
@@ -359,6 +527,12 @@ def run_ours(args, rank, world, local):
     e2e_value = world * 2 * n / (e2e_ms * 1e-3) / GB
     torch.cuda.synchronize(dev)
 
+    # ---- every workload's quantize kernel (N = 1 only) ----
+    per_cfg = None
+    if world == 1 and not args.no_per_config:
+        per_cfg = per_config_leg(nv, torch, dev, stream, measured_peak()[0],
+                                 resident={WORKLOAD: (x_np, (g, r, c))} if args.rows is None else None)
+
     # ---- CPU oracle on a bounded sample (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -382,7 +556,7 @@ def run_ours(args, rank, world, local):
                 "parallelism": f"dp{world} (independent tensors, no collective on the data path)",
             },
             "roofline": {
-                "kernel": "quantize_kernel<four_over_six, mse, codes>", "bound": "hbm",
+                "kernel": "quantize_grouped_kernel<four_over_six, mse, codes>", "bound": "hbm",
                 "achieved": round(ach["quantize"], 1), "peak": peak, "unit": "GB/s",
                 "frac": round(ach["quantize"] / peak, 4), "peak_kind": peak_kind,
                 "bytes_per_launch": ab["quantize"], "traffic": traffic,
@@ -401,8 +575,10 @@ def run_ours(args, rank, world, local):
             "gpu_launches": launches,
             "clocks": clocks.summary(),
         }
+        if per_cfg is not None:
+            line["per_config"] = per_cfg
         if cpu is not None:
-            line["cpu_baseline"] = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}
+            line["cpu_baseline"] = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample", "single_thread")}
         print(json.dumps(line), flush=True)
 
 

@@ -3,6 +3,7 @@
 // beyond a per-device cache of launch limits.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 
@@ -100,6 +101,29 @@ nvfp4_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// Grid of the grouped quantize kernel: gy rows of CTAs walk the groups (g = y, y + gy, ...),
+// gx CTAs share each group's warp tiles (64 blocks each). With `full` resident CTAs, pick the gy
+// that minimises the longest CTA's work, rounds x (tiles per warp + one tile's worth of
+// per-group setup), so that e.g. 64 experts on 296 CTA slots get 32 x 9 CTAs, not 64 x 4.
+dim3 grouped_grid(int64_t full, int64_t groups, int64_t bpg) {
+    constexpr int64_t kWarps = kThreads / 32;
+    const int64_t ntiles = (bpg + 63) / 64;
+    const int64_t xmax = std::max<int64_t>(1, (ntiles + kWarps - 1) / kWarps);
+    const int64_t gymax = std::max<int64_t>(1, std::min<int64_t>(groups, std::min<int64_t>(full, 65535)));
+    int64_t best_gx = 1, best_gy = 1, best = INT64_MAX;
+    for (int64_t gy = 1; gy <= gymax; ++gy) {
+        const int64_t gx = std::max<int64_t>(1, std::min<int64_t>(full / gy, xmax));
+        const int64_t rounds = (groups + gy - 1) / gy;
+        const int64_t t = rounds * ((ntiles + gx * kWarps - 1) / (gx * kWarps) + 1);
+        if (t < best) {
+            best = t;
+            best_gx = gx;
+            best_gy = gy;
+        }
+    }
+    return dim3(static_cast<unsigned>(best_gx), static_cast<unsigned>(best_gy));
+}
+
 template <bool FOUR, int RULE, bool FQ>
 nvfp4_status launch_quant(const nvfp4::QuantParams& p, cudaStream_t stream) {
     const int64_t bpg = p.gdiv.bpg;
@@ -107,13 +131,8 @@ nvfp4_status launch_quant(const nvfp4::QuantParams& p, cudaStream_t stream) {
     if (grouped) {
         // CTAs work inside one group at a time, with the group's scale table in shared memory
         auto kernel = nvfp4::quantize_grouped_kernel<FOUR, RULE, FQ>;
-        const int64_t full = static_cast<int64_t>(sm_count()) * ctas_per_sm(kernel);
-        const int64_t gy = p.groups < 65535 ? p.groups : 65535;
-        int64_t gx = full / gy;
-        const int64_t need = (bpg + kThreads - 1) / kThreads;
-        if (gx > need) gx = need;
-        if (gx < 1) gx = 1;
-        kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), kThreads, 0, stream>>>(p);
+        const dim3 grid = grouped_grid(static_cast<int64_t>(sm_count()) * ctas_per_sm(kernel), p.groups, bpg);
+        kernel<<<grid, kThreads, 0, stream>>>(p);
     } else {
         auto kernel = nvfp4::quantize_kernel<FOUR, RULE, FQ>;
         const unsigned grid = grid_for(kernel, p.nblocks);
@@ -135,12 +154,8 @@ nvfp4_status dispatch_quant(nvfp4_mode mode, nvfp4_rule rule, const nvfp4::Quant
 template <bool FOUR, int RULE>
 nvfp4_status launch_quant_gemm(const nvfp4::QuantParams& p, cudaStream_t stream) {
     auto kernel = nvfp4::quantize_grouped_kernel<FOUR, RULE, false, true>;
-    const int64_t full = static_cast<int64_t>(sm_count()) * ctas_per_sm(kernel);
-    int64_t gx = full;
-    const int64_t need = (p.nblocks + kThreads - 1) / kThreads;
-    if (gx > need) gx = need;
-    if (gx < 1) gx = 1;
-    kernel<<<dim3(static_cast<unsigned>(gx), 1u), kThreads, 0, stream>>>(p);
+    kernel<<<grouped_grid(static_cast<int64_t>(sm_count()) * ctas_per_sm(kernel), 1, p.nblocks), kThreads, 0,
+             stream>>>(p);
     return launch_status();
 }
 

@@ -491,3 +491,21 @@ def test_p13_four_over_six_reduces_to_single_candidate_runs(rule):
     for k in ("codes", "scales", "tscale", "choice"):
         assert np.array_equal(s6[k], s6b[k])
     assert not s6["choice"].any()
+
+
+def test_row_ranges_quantize_like_the_whole_tensor():
+    """Blocks are independent once the tensor scale is fixed ([FOS] Adaptive block scaling
+    algorithm: each block picks its own candidate), so row ranges quantized with the whole
+    tensor's amax give the same codes, scales and choice bits as one call (the multi-threaded
+    CPU baseline depends on this). 48 blocks per row keep every range on a choice-byte
+    boundary."""
+    from nvfp4_block_scaled_13_b200 import synth
+
+    x, (g, r, c) = synth.make("c3", rows=37, cols=768)
+    a = O.amax(x, 1, r, c)
+    whole = O.quantize(x, 1, r, c, a, 1, 2)
+    parts = [(0, 5), (5, 6), (6, 30), (30, 37)]
+    got = [O.quantize(np.ascontiguousarray(x[lo * c:hi * c]), 1, hi - lo, c, a, 1, 2) for lo, hi in parts]
+    for k in ("codes", "scales", "choice"):
+        assert np.array_equal(np.concatenate([q[k] for q in got]), whole[k]), k
+    assert all(np.array_equal(q["tscale"], whole["tscale"]) for q in got)
