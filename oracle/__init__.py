@@ -210,3 +210,33 @@ def qad_kl(teacher: np.ndarray, student: np.ndarray, rows: int, vocab: int, tau:
     g = np.zeros(rows * vocab, np.float64) if with_grad else None
     lib().nvo_qad_kl(_ptr(t), _ptr(s), rows, vocab, float(tau), float(grad_scale), _ptr(kl), _ptr(g))
     return kl, g
+
+
+def unpack_e2m1(codes: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """Packed E2M1 codes [rows, cols/2] bytes (element 2j in the low nibble, 2j + 1 in the
+    high nibble) -> the 4-bit codes [rows, cols] as uint8."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8).reshape(rows, cols // 2)
+    out = np.empty((rows, cols), np.uint8)
+    out[:, 0::2] = c & 0x0F
+    out[:, 1::2] = c >> 4
+    return out
+
+
+def gemm_nvfp4(a_codes, a_scales, a_alpha, b_codes, b_scales, b_alpha, m: int, n: int, k: int) -> np.ndarray:
+    """Y[m, n] = a_alpha * b_alpha * sum_k A[m, k] * B[n, k] in binary64, the product that a
+    block-scaled FP4 tensor-core GEMM forms from two NVFP4 operands ("Four Over Six",
+    Implementation details: NVFP4 operands on Blackwell's FP4 tensor cores; Problem definition:
+    a stored value is v(code) * E4M3 block scale * FP32 tensor scale). A[m, k] =
+    v(code) * f32(scale of block k / 16), exact in binary64; codes are [rows, k/2] bytes with
+    element 2j in the low nibble, scales row-major [rows, k/16] E4M3 bytes. The sum over k is
+    a float64 matrix product (exact for the sizes the tests use: every term has at most 7
+    significant bits); the tensor scales multiply once at the end."""
+    v = e2m1_to_f32(np.arange(16)).astype(np.float64)           # the oracle's decodes, as tables
+    sv = e4m3_to_f32(np.arange(256)).astype(np.float64)
+
+    def values(codes, scales, rows):
+        x = v[unpack_e2m1(codes, rows, k)]
+        return x * np.repeat(sv[np.asarray(scales, np.uint8).reshape(rows, k // 16)], 16, axis=1)
+
+    a, b = values(a_codes, a_scales, m), values(b_codes, b_scales, n)
+    return (a @ b.T) * (float(np.float32(a_alpha)) * float(np.float32(b_alpha)))
