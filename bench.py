@@ -175,7 +175,7 @@ def ncu_traffic(kernel: str):
     if not os.path.exists(path):
         return None
     src = b""
-    for f in ("kernels.cuh", "ptx.cuh"):
+    for f in ("kernels.cuh", "block.cuh", "ptx.cuh"):
         with open(os.path.join(ROOT, "nvfp4_block_scaled_13_b200", "csrc", f), "rb") as fh:
             src += fh.read()
     h = hashlib.sha256(src).hexdigest()[:16]

@@ -175,6 +175,39 @@ NVFP4_API nvfp4_status nvfp4_quantize_gemm(const uint16_t* x, int64_t rows, int6
  * magnitude (tests/test_gpu_5_qad_kl.py states the bounds). tau must be finite and > 0,
  * grad_scale finite (else NVFP4_ERR_VALUE); vocab >= 1; logits must be finite. rows == 0 does
  * nothing. One kernel; a second read of each row when grad is requested. */
+/* Bit set in a GEMM's status word when one of the kernel's bounded waits for the tensor core
+ * timed out (about two seconds); the kernel then stops, frees its tensor memory and leaves y
+ * partly written. */
+#define NVFP4_GEMM_TIMEOUT 1u
+
+/* Block-scaled FP4 GEMM on the 5th-generation tensor cores (tcgen05, kind::mxf4nvf4 with
+ * 16-element E4M3 scale blocks): y[m, n] = alpha_x * alpha_w * sum_k Xq[m, k] * Wq[n, k], FP32,
+ * row-major. NVFP4 operands run on Blackwell's FP4 tensor cores ("Four Over Six",
+ * Implementation details; "NVIDIA Model Optimizerを用いたNemotron 3.5 Lightning NVFP4とQADの開発",
+ * NVFP4 section). Both operands are K-major NVFP4 as written by nvfp4_quantize_gemm:
+ *   x_codes [m, k/2], x_scales tiled, x_tscale [1] alpha_x      (in, device)
+ *   w_codes [n, k/2], w_scales tiled, w_tscale [1] alpha_w      (in, device)
+ *   y       [m, n] FP32                                          (out, device)
+ *   status  nullable device word; NVFP4_GEMM_TIMEOUT is or-ed in on a timed-out wait (in/out)
+ * m must be a multiple of 128, n and k multiples of 256 (else NVFP4_ERR_SHAPE); codes,
+ * scales and y 16-byte aligned; the tensor-map encoder of the driver must be available (else
+ * NVFP4_ERR_CUDA). The accumulation is FP32 inside the tensor core, so y agrees
+ * with the exact product to within FP32 accumulation error, not bit for bit. */
+NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const float* x_tscale,
+                                  const uint8_t* w_codes, const uint8_t* w_scales, const float* w_tscale,
+                                  int64_t m, int64_t n, int64_t k, float* y, uint32_t* status,
+                                  cudaStream_t stream);
+
+/* The same GEMM with the activation operand quantized inside the kernel's prologue from BF16
+ * x [m, k] (32-byte aligned) with its amax x_amax [1] (device), in `mode` under `rule`,
+ * exactly as nvfp4_quantize_gemm would quantize it (the pages apply Four Over Six to the
+ * activations: "Four Over Six", Results). y equals nvfp4_gemm on nvfp4_quantize_gemm's
+ * output bit for bit. */
+NVFP4_API nvfp4_status nvfp4_gemm_quantize_x(const uint16_t* x, const float* x_amax, nvfp4_mode mode,
+                                             nvfp4_rule rule, const uint8_t* w_codes, const uint8_t* w_scales,
+                                             const float* w_tscale, int64_t m, int64_t n, int64_t k, float* y,
+                                             uint32_t* status, cudaStream_t stream);
+
 NVFP4_API nvfp4_status nvfp4_qad_kl(const uint16_t* teacher, const uint16_t* student, int64_t rows, int64_t vocab,
                                     float tau, float grad_scale, float* kl, uint16_t* grad, cudaStream_t stream);
 

@@ -23,10 +23,12 @@ __all__ = [
     "load", "library_path", "Nvfp4Error",
     "SCALE6", "FOUR_OVER_SIX", "RULE_MAXERR", "RULE_MAE", "RULE_MSE",
     "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_quantize_gemm", "nvfp4_qad_kl",
-    "nvfp4_status_string", "nvfp4_version",
+    "nvfp4_gemm", "nvfp4_gemm_quantize_x", "GEMM_TIMEOUT", "nvfp4_status_string", "nvfp4_version",
     "Quantized", "amax", "quantize", "fakequant", "dequantize", "quantize_for_gemm", "gemm_scale_bytes",
-    "qad_kl", "fakequant_ste",
+    "qad_kl", "fakequant_ste", "gemm", "gemm_quantize_x",
 ]
+
+GEMM_TIMEOUT = 1   # bit of a GEMM's status word: a bounded wait for the tensor core timed out
 
 SCALE6, FOUR_OVER_SIX = 0, 1
 RULE_MAXERR, RULE_MAE, RULE_MSE = 0, 1, 2
@@ -63,8 +65,10 @@ def load():
         L.nvfp4_fakequant.argtypes = [vp, i64, i64, i64, vp, i32, i32, vp, vp, vp]
         L.nvfp4_quantize_gemm.argtypes = [vp, i64, i64, vp, i32, i32, vp, vp, vp, vp, vp]
         L.nvfp4_qad_kl.argtypes = [vp, vp, i64, i64, ctypes.c_float, ctypes.c_float, vp, vp, vp]
+        L.nvfp4_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp]
+        L.nvfp4_gemm_quantize_x.argtypes = [vp, vp, i32, i32, vp, vp, vp, i64, i64, i64, vp, vp, vp]
         for f in (L.nvfp4_amax, L.nvfp4_quantize, L.nvfp4_dequantize, L.nvfp4_fakequant, L.nvfp4_quantize_gemm,
-                  L.nvfp4_qad_kl):
+                  L.nvfp4_qad_kl, L.nvfp4_gemm, L.nvfp4_gemm_quantize_x):
             f.restype = i32
         L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
         L.nvfp4_version.argtypes, L.nvfp4_version.restype = [], i32
@@ -130,6 +134,18 @@ def nvfp4_dequantize(codes, scales, tscale, groups, rows, cols, y, stream=None):
 def nvfp4_fakequant(x, groups, rows, cols, amax, mode, rule, y, choice=None, stream=None):
     _check(load().nvfp4_fakequant(_ptr(x), groups, rows, cols, _ptr(amax), _mode(mode), _rule(rule),
                                   _ptr(y), _ptr(choice), _stream(stream)), "nvfp4_fakequant")
+
+
+def nvfp4_gemm(x_codes, x_scales, x_tscale, w_codes, w_scales, w_tscale, m, n, k, y, status=None, stream=None):
+    _check(load().nvfp4_gemm(_ptr(x_codes), _ptr(x_scales), _ptr(x_tscale), _ptr(w_codes), _ptr(w_scales),
+                             _ptr(w_tscale), m, n, k, _ptr(y), _ptr(status), _stream(stream)), "nvfp4_gemm")
+
+
+def nvfp4_gemm_quantize_x(x, x_amax, mode, rule, w_codes, w_scales, w_tscale, m, n, k, y, status=None,
+                          stream=None):
+    _check(load().nvfp4_gemm_quantize_x(_ptr(x), _ptr(x_amax), _mode(mode), _rule(rule), _ptr(w_codes),
+                                        _ptr(w_scales), _ptr(w_tscale), m, n, k, _ptr(y), _ptr(status),
+                                        _stream(stream)), "nvfp4_gemm_quantize_x")
 
 
 def nvfp4_quantize_gemm(x, rows, cols, amax, mode, rule, codes, scales, tscale, choice=None, stream=None):
@@ -245,6 +261,38 @@ def quantize_for_gemm(x, mode="four_over_six", rule="mse", amax_values=None, wit
     choice = torch.empty(max(1, (nb + 7) // 8), dtype=torch.uint8, device=dev) if with_choice else None
     nvfp4_quantize_gemm(x, rows, cols, amax_values, mode, rule, codes, scales, tscale, choice, stream)
     return codes, scales, tscale, choice
+
+
+def gemm(xq, wq, stream=None):
+    """y = Xq Wq^T (FP32) of two operands returned by quantize_for_gemm, on the FP4 tensor
+    cores. Raises if the kernel reports a timed-out wait."""
+    import torch
+
+    (xc, xs, xt, _), (wc, ws, wt, _) = xq, wq
+    m, n, k = xc.shape[0], wc.shape[0], 2 * xc.shape[1]
+    y = torch.empty((m, n), dtype=torch.float32, device=xc.device)
+    status = torch.zeros(1, dtype=torch.int32, device=xc.device)
+    nvfp4_gemm(xc, xs, xt, wc, ws, wt, m, n, k, y, status, stream)
+    if int(status.item()) & GEMM_TIMEOUT:
+        raise Nvfp4Error("nvfp4_gemm: a wait for the tensor core timed out")
+    return y
+
+
+def gemm_quantize_x(x, wq, mode="four_over_six", rule="mse", amax_values=None, stream=None):
+    """y = Q(x) Wq^T (FP32), x [m, k] BF16 quantized inside the GEMM's prologue."""
+    import torch
+
+    wc, ws, wt, _ = wq
+    m, k = x.shape
+    n = wc.shape[0]
+    if amax_values is None:
+        amax_values = amax(x, 1, stream)
+    y = torch.empty((m, n), dtype=torch.float32, device=x.device)
+    status = torch.zeros(1, dtype=torch.int32, device=x.device)
+    nvfp4_gemm_quantize_x(x, amax_values, mode, rule, wc, ws, wt, m, n, k, y, status, stream)
+    if int(status.item()) & GEMM_TIMEOUT:
+        raise Nvfp4Error("nvfp4_gemm_quantize_x: a wait for the tensor core timed out")
+    return y
 
 
 def qad_kl(teacher, student, tau: float = 1.0, grad_scale=None, with_grad: bool = True, stream=None):

@@ -1,0 +1,260 @@
+// block.cuh — per-block arithmetic of the NVFP4 quantizer (sm_100a), shared by the
+// quantizer kernels and the prologue of the block-scaled FP4 GEMM.
+//
+// Layout in HBM: x is a flat array of 16-element BF16 blocks (32 bytes each); block b of the
+// flat index belongs to group b / blocks_per_group. Per block the quantizer writes 8 bytes of
+// codes, 1 byte of E4M3 scale and 1 choice bit; the fake-quant variant writes 32 bytes of BF16.
+//
+// The quantizer is issue-bound, not memory-bound, so the per-block arithmetic is kept small:
+//  - block scales without a division: lo = RN(m * RN(RN(1/beta) (1 - 2^-20))) and
+//    hi = RN(m * RN(RN(1/beta) (1 + 2^-20))) bracket the exact quotient RN(m/beta), so when
+//    E4M3(lo) == E4M3(hi) the scale is proven; otherwise (rare) the exact division decides;
+//  - the decode scale d = RN(f32(s) * alpha) and its reciprocal for every E4M3 code s come
+//    from a 128-entry table per group in shared memory (kernels whose CTAs work inside one
+//    group at a time), or are computed per block (the generic kernel);
+//  - packed .f32x2 arithmetic, three-input max, and 32-bit in-group indices.
+#pragma once
+
+#include <float.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+constexpr int kThreads = 256;
+
+enum Rule : int { kMaxErr = 0, kMae = 1, kMse = 2 };
+
+// Group lookup for the generic kernel: g = b / blocks_per_group. Division by an invariant
+// integer with a precomputed multiplier (exact for b < 2^31); the 64-bit quotient otherwise.
+struct GroupDiv {
+    int64_t bpg;          // blocks per group
+    uint32_t mul;         // ceil(2^(31 + l) / bpg), l = ceil(log2 bpg)
+    uint32_t shift;       // l - 1
+    int mode;             // 0: single group, 1: bpg == 1, 2: multiplier, 3: 64-bit divide
+
+    __device__ __forceinline__ int64_t operator()(int64_t b) const {
+        switch (mode) {
+            case 0: return 0;
+            case 1: return b;
+            case 2: return static_cast<int64_t>(__umulhi(static_cast<uint32_t>(b), mul) >> shift);
+            default: return b / bpg;
+        }
+    }
+};
+
+struct QuantParams {
+    const uint16_t* x;
+    const float* amax;
+    uint8_t* codes;      // codes output (quantize) or nullptr (fake-quant)
+    uint8_t* scales;
+    float* tscale;
+    uint8_t* choice;     // nullable
+    uint16_t* y;         // fake-quant output or nullptr
+    int64_t nblocks;
+    int64_t choice_bytes;
+    int64_t groups;
+    GroupDiv gdiv;
+    // tiled scale layout of block-scaled GEMM operands (one group, a [rows, 16 * bpr] matrix):
+    // blocks per row, multiply-shift divisor for it (exact below 2^31), 4-column tiles per row
+    uint32_t bpr, bpr_mul, bpr_shift, n_ct;
+};
+
+struct DequantParams {
+    const uint8_t* codes;
+    const uint8_t* scales;
+    const float* tscale;
+    uint16_t* y;
+    int64_t nblocks;
+    int64_t groups;
+    GroupDiv gdiv;
+};
+
+// ---- small helpers ------------------------------------------------------------------------------
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ float recip_clamped(float d) {
+    return d > 0.0f ? fminf(__frcp_rn(d), FLT_MAX) : 0.0f;
+}
+
+// Per-group constants: alpha = amax / (6 M), beta_K = K * alpha, and the bracket factors
+// yl_K = RN(RN(1/beta_K) * (1 - 2^-20)), yh_K = RN(RN(1/beta_K) * (1 + 2^-20)) used to bracket
+// the block-scale quotients (valid when both betas lie in [2^-125, 2^125], so that every
+// factor is a normal number).
+struct GroupCtx {
+    float alpha, beta6, beta4, yl6, yh6, yl4, yh4;
+    bool fast;
+};
+
+template <bool FOUR>
+__device__ __forceinline__ GroupCtx make_group(float amax, float six_m) {
+    GroupCtx c;
+    c.alpha = __fdiv_rn(amax, six_m);
+    c.beta6 = __fmul_rn(6.0f, c.alpha);
+    c.beta4 = __fmul_rn(4.0f, c.alpha);
+    const float lo = FOUR ? c.beta4 : c.beta6;
+    c.fast = lo >= 0x1p-125f && c.beta6 <= 0x1p125f;
+    constexpr float kLo = 1.0f - 0x1p-20f, kHi = 1.0f + 0x1p-20f;
+    const float y6 = c.fast ? __frcp_rn(c.beta6) : 0.0f, y4 = c.fast ? __frcp_rn(c.beta4) : 0.0f;
+    c.yl6 = __fmul_rn(y6, kLo);
+    c.yh6 = __fmul_rn(y6, kHi);
+    c.yl4 = __fmul_rn(y4, kLo);
+    c.yh4 = __fmul_rn(y4, kHi);
+    return c;
+}
+
+// E4M3(RN(m / beta_6)) in the low byte and E4M3(RN(m / beta_4)) in the high byte.
+// lo = RN(m * yl) and hi = RN(m * yh) carry three roundings of at most 2^-24 each on top of
+// the factors 1 -+ 2^-20, so lo < m/beta * (1 - 2^-21) < RN(m / beta) < hi whenever the
+// products are normal; below 2^-126 every one of them converts to E4M3 zero, and an overflow
+// saturates to 448 like the quotient it bounds. E4M3 rounding is monotone, so equal
+// conversions of lo and hi are the exact scale. Near a rounding boundary (about one block in
+// 2^15), or outside the factors' valid range, the exact division decides.
+template <bool FOUR>
+__device__ __forceinline__ uint32_t block_scales(float m, const GroupCtx& c) {
+    if (c.fast) {
+        if (FOUR) {
+            const float2 lo = mul2(make_float2(m, m), make_float2(c.yl6, c.yl4));
+            const float2 hi = mul2(make_float2(m, m), make_float2(c.yh6, c.yh4));
+            const uint32_t wl = e4m3x2(lo.x, lo.y), wh = e4m3x2(hi.x, hi.y);
+            if (wl == wh) return wl;
+        } else {
+            const float2 b = mul2(make_float2(m, m), make_float2(c.yl6, c.yh6));
+            const uint32_t b6 = e4m3x2(b.x, b.y);
+            if ((b6 & 0xFFu) == (b6 >> 8)) return b6 & 0xFFu;
+        }
+    }
+    const float t6 = c.beta6 > 0.0f ? __fdiv_rn(m, c.beta6) : 0.0f;
+    const float t4 = FOUR ? (c.beta4 > 0.0f ? __fdiv_rn(m, c.beta4) : 0.0f) : 0.0f;
+    return e4m3x2(t6, t4);
+}
+
+// Decode scale and encode factor for E4M3 code s: d = RN(f32(s) * alpha), r = min(1/d, FLT_MAX).
+__device__ __forceinline__ float2 scale_entry(uint32_t s, float alpha) {
+    const float d = __fmul_rn(e4m3x2_to_float2(s).x, alpha);
+    return make_float2(d, recip_clamped(d));
+}
+
+// One candidate (target maximum K) of one block: its codes, their exact values as f16x2
+// words, and the rule's error. e_i = x_i - v_i * d is one fused multiply-add (the exact
+// difference, rounded once). MAE/MSE keep two running sums, one over even and one over odd
+// element indices (for MSE the two lanes of a packed pair), added at the end.
+template <int RULE>
+__device__ __forceinline__ float candidate(const float2 (&x)[8], float r, float d, uint32_t& c_lo,
+                                           uint32_t& c_hi, uint32_t (&h)[8]) {
+    const float2 rr = make_float2(r, r), nd = make_float2(-d, -d);
+    float2 y[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = mul2(x[j], rr);
+    c_lo = e2m1x8_and_decode(y[0], y[1], y[2], y[3], h[0], h[1], h[2], h[3]);
+    c_hi = e2m1x8_and_decode(y[4], y[5], y[6], y[7], h[4], h[5], h[6], h[7]);
+    float2 acc = make_float2(0.0f, 0.0f);
+    float emax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float2 e = fma2(f16x2_to_float2(h[j]), nd, x[j]);
+        if (RULE == kMse) {
+            acc = fma2(e, e, acc);
+        } else if (RULE == kMae) {
+            acc.x = __fadd_rn(acc.x, fabsf(e.x));
+            acc.y = __fadd_rn(acc.y, fabsf(e.y));
+        } else {
+            emax = max3(emax, fabsf(e.x), fabsf(e.y));
+        }
+    }
+    return RULE == kMaxErr ? emax : __fadd_rn(acc.x, acc.y);
+}
+
+// Quantize the block in `w` (eight BF16 pairs) into registers: the kept candidate's codes
+// (clo: elements 0-7, chi: 8-15, element 2j in the low nibble), its E4M3 scale s and decode
+// scale d, and (FQ) its values as f16x2 words in h. Returns whether target 4 was kept.
+// TABLE: d and 1/d come from `tab`.
+template <bool FOUR, int RULE, bool FQ, bool TABLE>
+__device__ __forceinline__ bool quantize_block_regs(const uint32_t (&w)[8], const GroupCtx& gc, const float2* tab,
+                                                    uint32_t& clo, uint32_t& chi, uint32_t& s, float& dsel,
+                                                    uint32_t (&h)[8]) {
+    float2 x[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = unpack_bf16x2(w[j]);
+    // max over {0, |x_i|}: depth-3 tree of 3-input max (the same value as a running max)
+    const float m01 = max3(0.0f, fabsf(x[0].x), fabsf(x[0].y));
+    const float m02 = max3(fabsf(x[1].x), fabsf(x[1].y), fabsf(x[2].x));
+    const float m03 = max3(fabsf(x[2].y), fabsf(x[3].x), fabsf(x[3].y));
+    const float m04 = max3(fabsf(x[4].x), fabsf(x[4].y), fabsf(x[5].x));
+    const float m05 = max3(fabsf(x[5].y), fabsf(x[6].x), fabsf(x[6].y));
+    const float m06 = max3(fabsf(x[7].x), fabsf(x[7].y), 0.0f);
+    const float m = fmaxf(max3(m01, m02, m03), max3(m04, m05, m06));
+    const uint32_t s2 = block_scales<FOUR>(m, gc);
+    const uint32_t i6 = __byte_perm(s2, 0u, 0x4440), i4 = __byte_perm(s2, 0u, 0x4441);
+    const float2 e6 = TABLE ? tab[i6] : scale_entry(i6, gc.alpha);
+    const float err6 = candidate<RULE>(x, e6.y, e6.x, clo, chi, h);
+    s = i6;
+    dsel = e6.x;
+    bool four = false;
+    if (FOUR) {
+        const float2 e4 = TABLE ? tab[i4] : scale_entry(i4, gc.alpha);
+        uint32_t c4lo, c4hi, h4[8];
+        const float err4 = candidate<RULE>(x, e4.y, e4.x, c4lo, c4hi, h4);
+        four = err4 < err6;   // ties keep target 6
+        if (four) {
+            clo = c4lo;
+            chi = c4hi;
+            s = i4;
+            dsel = e4.x;
+        }
+        if (FQ) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) h[j] = four ? h4[j] : h[j];
+        }
+    }
+    return four;
+}
+
+// Quantize the block in `w` and store its codes + scale (or fake-quant BF16); returns whether
+// target 4 was kept. ok = false (a lane past the end of the group) computes but stores nothing
+// and returns false.
+template <bool FOUR, int RULE, bool FQ, bool TABLE>
+__device__ __forceinline__ bool quantize_block(const uint32_t (&w)[8], const GroupCtx& gc, const float2* tab,
+                                               uint8_t* codes8, uint8_t* scale1, uint16_t* y16, bool ok = true) {
+    uint32_t clo, chi, s, h[8];
+    float dsel;
+    const bool four = quantize_block_regs<FOUR, RULE, FQ, TABLE>(w, gc, tab, clo, chi, s, dsel, h);
+    if (FQ) {   // q = RN(v * d) of the kept candidate, rounded to BF16
+        const float2 dd = make_float2(dsel, dsel);
+        uint32_t out[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) out[j] = bf16x2(mul2(f16x2_to_float2(h[j]), dd));
+        if (ok) st32(y16, out);
+    } else if (ok) {
+        st8(codes8, clo, chi);
+        *scale1 = static_cast<uint8_t>(s);
+    }
+    return four && ok;
+}
+
+// Byte offset of local block a's scale in the tiled layout: 128-row x 4-column tiles of 512
+// bytes, tile (row / 128, col / 4) at ((row / 128) * n_ct + col / 4) * 512, and inside a tile
+// row r, column c at (r % 32) * 16 + (r / 32) * 4 + c.
+__device__ __forceinline__ uint32_t tiled_scale_offset(uint32_t a, const QuantParams& p) {
+    const uint32_t row = p.bpr == 1u ? a : __umulhi(a, p.bpr_mul) >> p.bpr_shift;
+    const uint32_t col = a - row * p.bpr;
+    return (((row >> 7) * p.n_ct + (col >> 2)) << 9) + ((row & 31u) << 4) + (((row >> 5) & 3u) << 2) + (col & 3u);
+}
+
+// Store one warp's 32 choice bits (the word starting at flat block `first`, a multiple of 32).
+__device__ __forceinline__ void store_choice(uint8_t* choice, int64_t choice_bytes, int64_t first, uint32_t bits) {
+    const int64_t byte0 = first >> 3;
+    if (byte0 + 4 <= choice_bytes) {
+        *reinterpret_cast<uint32_t*>(choice + byte0) = bits;
+    } else {
+        for (int k = 0; byte0 + k < choice_bytes; ++k) choice[byte0 + k] = static_cast<uint8_t>(bits >> (8 * k));
+    }
+}
+
+}  // namespace nvfp4

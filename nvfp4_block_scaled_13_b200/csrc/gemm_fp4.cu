@@ -1,0 +1,492 @@
+// gemm_fp4.cu — block-scaled FP4 GEMM on the 5th-generation tensor cores of sm_100a:
+//
+//     Y[m, n] = alpha_x * alpha_w * sum_k Xq[m, k] * Wq[n, k]        (FP32 out, row-major)
+//
+// with NVFP4 operands: E2M1 values, one E4M3 scale per 16 consecutive elements along K and
+// one FP32 tensor scale per operand ("Four Over Six", Problem definition and Implementation
+// details: NVFP4 weights and activations run on Blackwell's FP4 tensor cores, and applying
+// 4/6 to the activations alone recovers most of the accuracy). The activation operand Xq
+// either comes in quantized (codes + scales in the tiled layout of nvfp4_quantize_gemm), or is
+// quantized from BF16 inside this kernel, in the GEMM's prologue, with the same per-block
+// arithmetic as nvfp4_quantize (scale-6 or Four Over Six under a max / MAE / MSE rule).
+//
+// One CTA computes a 128 x 256 tile of Y with warp-specialised roles over a 4-stage ring of
+// K slices (256 elements: four MMAs of K = 64) in shared memory:
+//   warp 0 (one lane)  TMA: B codes (and A codes when pre-quantized) as 128-byte swizzled
+//                      tiles, and the operands' 512-byte scale tiles as bulk copies, all
+//                      completing on the stage's "full" mbarrier;
+//   warps 2-7          (prologue variant) quantize the stage's 128 x 256 BF16 activations
+//                      into the swizzled A tile and its scale tiles, then arrive on "full";
+//   warp 1 (one lane)  waits for "full", copies the scale tiles into tensor memory
+//                      (tcgen05.cp.32x128b.warpx4), issues four
+//                      tcgen05.mma.kind::mxf4nvf4.block_scale.block16 into the FP32
+//                      accumulator in tensor memory, and commits them to the stage's "empty"
+//                      mbarrier, which releases the slot to the producers.
+// The epilogue (warps 0-3, one 32-lane quarter of tensor memory each) reads the accumulator
+// with tcgen05.ld and scales it by alpha_x * alpha_w. Every mbarrier wait is bounded: on
+// timeout the kernel records NVFP4_GEMM_TIMEOUT in the status word, every role stops, the
+// CTA frees its tensor memory and returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/nvfp4.h"
+#include "block.cuh"
+
+namespace {
+
+using namespace nvfp4;
+
+constexpr int kBM = 128, kBN = 256, kBK = 256;    // CTA tile and K slice (elements)
+constexpr int kStages = 4;
+constexpr int kQuantWarps = 6;                    // prologue variant: warps 2..7
+constexpr uint32_t kTmemCols = 512;
+// tensor memory: accumulator columns 0..255; per stage, A scales 4 x 4 columns from 256 and
+// B scales 4 x 8 columns from 320
+constexpr uint32_t kColSfa = 256, kColSfb = 320;
+// shared memory per stage: A codes 128 rows x 128 bytes, B codes 256 x 128 (128-byte
+// swizzled, 1024-byte aligned), A scale tiles 4 x 512 bytes, B scale tiles 8 x 512 bytes
+constexpr uint32_t kABytes = kBM * 128, kBBytes = kBN * 128;
+constexpr uint32_t kSfaBytes = 4 * 512, kSfbBytes = 8 * 512;
+constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;   // 55296, a multiple of 1024
+constexpr uint32_t kDynSmem = kStages * kStageBytes + 1024;                   // + alignment slack
+constexpr unsigned long long kWaitCycles = 4000000000ull;                     // about two seconds at 2 GHz
+
+// ---- PTX wrappers -------------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the mbarrier phase with the given parity to complete.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    const unsigned long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > kWaitCycles) return false;
+    }
+    return true;
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {   // whole warp
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {     // whole warp
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Shared-memory matrix descriptor, K-major without swizzle: core matrices of 8 rows x 16 bytes
+// (128 contiguous bytes); `lbo` = bytes between the two 16-byte K chunks of one MMA, `sbo` =
+// bytes between 8-row groups; version 1 (Blackwell) in bits 46-47, layout type 0.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    return d;
+}
+
+// The same for a K-major operand written with the 128-byte swizzle (TMA's SWIZZLE_128B):
+// rows of 128 bytes, 8-row atoms of 1024 bytes (SBO), layout type 2; the MMA with K offset j
+// (32 bytes each) starts 32 j bytes into the 1024-byte-aligned atom.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(1) << 16;
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// 2-D tiled TMA load of box {x, y} (x in bytes along K) into shared memory.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// Contiguous bulk copy (16-byte aligned, multiple of 16 bytes) into shared memory.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// Instruction descriptor of kind::mxf4nvf4 with 16-element E4M3 scale blocks: A and B E2M1
+// (format 1), both K-major, scale format E4M3 (0), M = 128, N = 256, dense, K = 64.
+constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kBN >> 3) << 17) |
+                            (static_cast<uint32_t>(kBM >> 4) << 24);
+
+// 32 rows x 16 bytes of scale factors (one 512-byte tile) -> 4 TMEM columns, replicated to
+// the four 32-lane quarters; row i of the tile lands in lane i (+32 q), column c, byte j
+// holding the scale of row i + 32 c and K block j of the MMA.
+__device__ __forceinline__ void tmem_copy_sf(uint32_t taddr, uint64_t desc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+
+__device__ __forceinline__ void mma_fp4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns of tensor memory -> 32 registers per thread.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void sts16(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void sts16b(uint32_t addr, uint16_t v) {
+    asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
+}  // namespace
+
+
+namespace {
+
+struct GemmParams {
+    const uint16_t* x;        // prologue variant: BF16 activations [m, k] (32-byte aligned)
+    const float* x_amax;      // prologue variant: amax of x, [1]
+    const uint8_t* x_scales;  // pre-quantized variant: tiled scales of x
+    const float* x_tscale;    // pre-quantized variant: alpha_x, [1]
+    const uint8_t* w_scales;  // tiled scales of w
+    const float* w_tscale;    // alpha_w, [1]
+    float* y;                 // [m, n]
+    uint32_t* status;         // nullable; NVFP4_GEMM_TIMEOUT is or-ed in on a timed-out wait
+    int64_t m, n, k;
+};
+
+// Grid (n / 256, m / 128). tmap_a / tmap_b: the codes of x / w as [rows, k/2] byte matrices,
+// boxes of 128 bytes x 128 (A) or 256 (B) rows, 128-byte swizzle (tmap_a unused when QUANT).
+template <bool QUANT, bool FOUR, int RULE>
+__global__ void __launch_bounds__(QUANT ? 256 : 128, 1)
+    gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                    const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full[kStages], empty[kStages], done;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ volatile uint32_t stop_sh;
+    __shared__ float2 tab[128];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t tn = blockIdx.x, tm = blockIdx.y;
+    const int64_t n_ct = p.k / 64;                   // scale tiles per 128 rows
+    const int nk = static_cast<int>(p.k / kBK);
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    const uint32_t full0 = smem_u32(&full[0]), empty0 = smem_u32(&empty[0]), done_bar = smem_u32(&done);
+
+    if (warp == 0) tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
+    if (tid == 32) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full0 + 8 * s, QUANT ? 1 + kQuantWarps : 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        mbar_init(done_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        stop_sh = 0;
+    }
+    GroupCtx gc{};
+    if (QUANT) {
+        constexpr float kSixM = FOUR ? 1536.0f : 2688.0f;
+        gc = make_group<FOUR>(__ldg(p.x_amax), kSixM);
+        if (tid < 128) tab[tid] = scale_entry(tid == 127 ? 126u : static_cast<uint32_t>(tid), gc.alpha);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    if (warp == 0) {
+        if (lane == 0) {   // producer: TMA and bulk copies into the ring
+            for (int ks = 0; ks < nk && !stop_sh; ++ks) {
+                const int s = ks % kStages;
+                const uint32_t u = static_cast<uint32_t>(ks / kStages);
+                if (ks >= kStages && !mbar_wait(empty0 + 8 * s, (u - 1) & 1)) {
+                    stop_sh = 1;
+                    break;
+                }
+                const uint32_t fb = full0 + 8 * s, sA = sbase + s * kStageBytes, sB = sA + kABytes;
+                const uint32_t sSFA = sB + kBBytes, sSFB = sSFA + kSfaBytes;
+                mbar_expect_tx(fb, (QUANT ? 0u : kABytes + kSfaBytes) + kBBytes + kSfbBytes);
+                if (!QUANT) {
+                    tma_load_2d(sA, &tmap_a, ks * (kBK / 2), static_cast<int32_t>(tm * kBM), fb);
+                    bulk_load(sSFA, p.x_scales + (tm * n_ct + 4 * ks) * 512, kSfaBytes, fb);
+                }
+                tma_load_2d(sB, &tmap_b, ks * (kBK / 2), static_cast<int32_t>(tn * kBN), fb);
+                bulk_load(sSFB, p.w_scales + (2 * tn * n_ct + 4 * ks) * 512, kSfbBytes / 2, fb);
+                bulk_load(sSFB + kSfbBytes / 2, p.w_scales + ((2 * tn + 1) * n_ct + 4 * ks) * 512, kSfbBytes / 2, fb);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {   // MMA issuer
+            for (int ks = 0; ks < nk && !stop_sh; ++ks) {
+                const int s = ks % kStages;
+                const uint32_t u = static_cast<uint32_t>(ks / kStages);
+                if (!mbar_wait(full0 + 8 * s, u & 1)) {
+                    stop_sh = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sA = sbase + s * kStageBytes, sB = sA + kABytes;
+                const uint32_t sSFA = sB + kBBytes, sSFB = sSFA + kSfaBytes;
+                const uint32_t ca = tmem + kColSfa + 16 * s, cb = tmem + kColSfb + 32 * s;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    tmem_copy_sf(ca + 4 * j, smem_desc(sSFA + 512 * j, 16, 128));
+                    tmem_copy_sf(cb + 8 * j, smem_desc(sSFB + 512 * j, 16, 128));                   // rows 0..127
+                    tmem_copy_sf(cb + 8 * j + 4, smem_desc(sSFB + kSfbBytes / 2 + 512 * j, 16, 128));   // 128..255
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    mma_fp4(tmem, smem_desc_sw128(sA + 32 * j), smem_desc_sw128(sB + 32 * j), kIdesc, ca + 4 * j,
+                            cb + 8 * j, (ks | j) != 0);
+                mma_commit(empty0 + 8 * s);
+            }
+            mma_commit(done_bar);   // arrives once every MMA issued above has completed
+        }
+    } else if (QUANT) {   // warps 2..7: quantize the stage's activations into the A tile
+        const int q = tid - 64;
+        for (int ks = 0; ks < nk && !stop_sh; ++ks) {
+            const int s = ks % kStages;
+            const uint32_t u = static_cast<uint32_t>(ks / kStages);
+            if (ks >= kStages) {
+                uint32_t ok = 1;
+                if (lane == 0) ok = mbar_wait(empty0 + 8 * s, (u - 1) & 1);
+                if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+                    stop_sh = 1;
+                    break;
+                }
+            }
+            const uint32_t sA = sbase + s * kStageBytes, sSFA = sA + kABytes + kBBytes;
+            // 1024 chunks of 32 elements (two blocks): chunk c = row c / 8, K chunk c % 8
+            for (int c = q; c < 1024; c += 32 * kQuantWarps) {
+                const int r = c >> 3, kc = c & 7;
+                const uint16_t* xs = p.x + (tm * kBM + r) * p.k + ks * kBK + kc * 32;
+                uint32_t w0[8], w1[8], c0lo, c0hi, c1lo, c1hi, s0, s1, h[8];
+                float d;
+                ld32_stream(xs, w0);
+                ld32_stream(xs + 16, w1);
+                quantize_block_regs<FOUR, RULE, false, true>(w0, gc, tab, c0lo, c0hi, s0, d, h);
+                quantize_block_regs<FOUR, RULE, false, true>(w1, gc, tab, c1lo, c1hi, s1, d, h);
+                // 128-byte swizzle: 16-byte chunk kc of row r at r * 128 + (kc ^ (r % 8)) * 16
+                sts16(sA + r * 128 + ((kc ^ (r & 7)) << 4), make_uint4(c0lo, c0hi, c1lo, c1hi));
+                // scale tile of MMA kc / 2: row r, K block j at (r % 32) * 16 + (r / 32) * 4 + j
+                sts16b(sSFA + (kc >> 1) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (kc & 1) * 2,
+                       static_cast<uint16_t>(s0 | (s1 << 8)));
+            }
+            fence_async_smem();   // the stores are read by the tensor core (async proxy)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full0 + 8 * s);
+        }
+    }
+    __syncthreads();   // every role has left its loop
+    if (tid == 0 && !mbar_wait(done_bar, 0)) stop_sh = 1;   // in-flight MMAs, bounded
+    __syncthreads();
+    tc_fence_after();
+    if (!stop_sh) {
+        if (warp < 4) {   // warp w reads tensor-memory lanes (rows) 32w..32w+31
+            const int64_t row = tm * kBM + 32 * warp + lane;
+            float* yr = p.y + row * p.n + tn * kBN;
+            const float alpha = (QUANT ? gc.alpha : __ldg(p.x_tscale)) * __ldg(p.w_tscale);
+#pragma unroll 1
+            for (int c = 0; c < kBN; c += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + c, r);
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4*>(yr + c + j) =
+                        make_float4(__uint_as_float(r[j]) * alpha, __uint_as_float(r[j + 1]) * alpha,
+                                    __uint_as_float(r[j + 2]) * alpha, __uint_as_float(r[j + 3]) * alpha);
+            }
+        }
+    } else if (tid == 0 && p.status != nullptr) {
+        atomicOr(p.status, NVFP4_GEMM_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---- host side -----------------------------------------------------------------------------------
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+// Tensor map of a [rows, row_bytes] byte matrix read in boxes of 128 bytes x box_rows rows
+// with the 128-byte swizzle.
+bool codes_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes, uint32_t box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+    const cuuint32_t box[2] = {128u, box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool QUANT, bool FOUR, int RULE>
+nvfp4_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& p, cudaStream_t stream) {
+    auto kernel = gemm_fp4_kernel<QUANT, FOUR, RULE>;
+    // per device, so set on every launch (cheap)
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(p.n / kBN), static_cast<unsigned>(p.m / kBM));
+    kernel<<<grid, QUANT ? 256 : 128, kDynSmem, stream>>>(ma, mb, p);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+bool aligned16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
+bool aligned4(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 3u) == 0; }
+
+nvfp4_status check_gemm_shape(int64_t m, int64_t n, int64_t k) {
+    if (m < 0 || n < 0 || k < 0) return NVFP4_ERR_SHAPE;
+    if (m % kBM || n % kBN || k % kBK) return NVFP4_ERR_SHAPE;
+    if (m / kBM > 65535 || n / kBN > 65535 || k > (int64_t(1) << 30) || m > (int64_t(1) << 31) ||
+        n > (int64_t(1) << 31))
+        return NVFP4_ERR_SHAPE;
+    return NVFP4_OK;
+}
+
+}  // namespace
+
+extern "C" nvfp4_status nvfp4_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const float* x_tscale,
+                                   const uint8_t* w_codes, const uint8_t* w_scales, const float* w_tscale,
+                                   int64_t m, int64_t n, int64_t k, float* y, uint32_t* status,
+                                   cudaStream_t stream) {
+    const nvfp4_status st = check_gemm_shape(m, n, k);
+    if (st != NVFP4_OK) return st;
+    if (m == 0 || n == 0) return NVFP4_OK;
+    if (!x_codes || !x_scales || !x_tscale || !w_codes || !w_scales || !w_tscale || !y) return NVFP4_ERR_NULL;
+    if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+        !aligned16(y) || !aligned4(x_tscale) || !aligned4(w_tscale) || !aligned4(status))
+        return NVFP4_ERR_ALIGN;
+    if (k == 0) return NVFP4_ERR_SHAPE;
+    CUtensorMap ma, mb;
+    if (!codes_map(&ma, x_codes, m, k / 2, kBM) || !codes_map(&mb, w_codes, n, k / 2, kBN)) return NVFP4_ERR_CUDA;
+    GemmParams p{};
+    p.x_scales = x_scales;
+    p.x_tscale = x_tscale;
+    p.w_scales = w_scales;
+    p.w_tscale = w_tscale;
+    p.y = y;
+    p.status = status;
+    p.m = m;
+    p.n = n;
+    p.k = k;
+    return launch_gemm<false, true, kMse>(ma, mb, p, stream);
+}
+
+extern "C" nvfp4_status nvfp4_gemm_quantize_x(const uint16_t* x, const float* x_amax, nvfp4_mode mode,
+                                              nvfp4_rule rule, const uint8_t* w_codes, const uint8_t* w_scales,
+                                              const float* w_tscale, int64_t m, int64_t n, int64_t k, float* y,
+                                              uint32_t* status, cudaStream_t stream) {
+    const nvfp4_status st = check_gemm_shape(m, n, k);
+    if (st != NVFP4_OK) return st;
+    if (mode != NVFP4_SCALE6 && mode != NVFP4_FOUR_OVER_SIX) return NVFP4_ERR_MODE;
+    if (rule != NVFP4_RULE_MAXERR && rule != NVFP4_RULE_MAE && rule != NVFP4_RULE_MSE) return NVFP4_ERR_RULE;
+    if (m == 0 || n == 0) return NVFP4_OK;
+    if (!x || !x_amax || !w_codes || !w_scales || !w_tscale || !y) return NVFP4_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(x) & 31u) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y) ||
+        !aligned4(x_amax) || !aligned4(w_tscale) || !aligned4(status))
+        return NVFP4_ERR_ALIGN;
+    if (k == 0) return NVFP4_ERR_SHAPE;
+    CUtensorMap ma, mb;
+    memset(&ma, 0, sizeof(ma));
+    if (!codes_map(&mb, w_codes, n, k / 2, kBN)) return NVFP4_ERR_CUDA;
+    GemmParams p{};
+    p.x = x;
+    p.x_amax = x_amax;
+    p.w_scales = w_scales;
+    p.w_tscale = w_tscale;
+    p.y = y;
+    p.status = status;
+    p.m = m;
+    p.n = n;
+    p.k = k;
+    if (mode == NVFP4_SCALE6) return launch_gemm<true, false, kMse>(ma, mb, p, stream);
+    switch (rule) {
+        case NVFP4_RULE_MAXERR: return launch_gemm<true, true, kMaxErr>(ma, mb, p, stream);
+        case NVFP4_RULE_MAE: return launch_gemm<true, true, kMae>(ma, mb, p, stream);
+        default: return launch_gemm<true, true, kMse>(ma, mb, p, stream);
+    }
+}

@@ -19,8 +19,9 @@ def header_functions(path):
 
 def test_header_declares_the_boundary():
     names = header_functions(os.path.join(ROOT, "include", "nvfp4.h"))
-    assert names == ["nvfp4_amax", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_qad_kl", "nvfp4_quantize",
-                     "nvfp4_quantize_gemm", "nvfp4_status_string", "nvfp4_version"]
+    assert names == ["nvfp4_amax", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_gemm", "nvfp4_gemm_quantize_x",
+                     "nvfp4_qad_kl", "nvfp4_quantize", "nvfp4_quantize_gemm", "nvfp4_status_string",
+                     "nvfp4_version"]
 
 
 def test_library_exports_every_declared_symbol():
@@ -86,6 +87,23 @@ A = 1 << 20          # 32-byte aligned
     (lambda L: L.nvfp4_qad_kl(A, A, 4, 8, 1.0, 1.0, None, None, None), 1),
     (lambda L: L.nvfp4_qad_kl(A + 1, A, 4, 8, 1.0, 1.0, A, None, None), 3),
     (lambda L: L.nvfp4_qad_kl(A, A, 4, 8, 1.0, 1.0, A + 2, None, None), 3),
+    # nvfp4_gemm(xc, xs, xt, wc, ws, wt, m, n, k, y, status, stream)
+    (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 100, 256, 256, A, None, None), 2),
+    (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 128, 256, 200, A, None, None), 2),
+    (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 128, 128, 256, A, None, None), 2),
+    (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 128, 256, 0, A, None, None), 2),
+    (lambda L: L.nvfp4_gemm(None, A, A, A, A, A, 128, 256, 256, A, None, None), 1),
+    (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 128, 256, 256, None, None, None), 1),
+    (lambda L: L.nvfp4_gemm(A + 8, A, A, A, A, A, 128, 256, 256, A, None, None), 3),
+    (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 128, 256, 256, A, A + 2, None), 3),
+    (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 0, 256, 256, None, None, None), 0),
+    # nvfp4_gemm_quantize_x(x, amax, mode, rule, wc, ws, wt, m, n, k, y, status, stream)
+    (lambda L: L.nvfp4_gemm_quantize_x(A, A, 2, 2, A, A, A, 128, 256, 256, A, None, None), 4),
+    (lambda L: L.nvfp4_gemm_quantize_x(A, A, 1, 3, A, A, A, 128, 256, 256, A, None, None), 5),
+    (lambda L: L.nvfp4_gemm_quantize_x(A, A, 1, 2, A, A, A, 128, 64, 256, A, None, None), 2),
+    (lambda L: L.nvfp4_gemm_quantize_x(None, A, 1, 2, A, A, A, 128, 256, 256, A, None, None), 1),
+    (lambda L: L.nvfp4_gemm_quantize_x(A, None, 1, 2, A, A, A, 128, 256, 256, A, None, None), 1),
+    (lambda L: L.nvfp4_gemm_quantize_x(A + 16, A, 1, 2, A, A, A, 128, 256, 256, A, None, None), 3),
     # nvfp4_fakequant(x, G, R, C, amax, mode, rule, y, choice, stream)
     (lambda L: L.nvfp4_fakequant(A, 1, 4, 32, A, 1, 2, None, None, None), 1),
     (lambda L: L.nvfp4_fakequant(A, 1, 4, 32, A, 7, 2, A, None, None), 4),
