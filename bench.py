@@ -166,6 +166,18 @@ def measured_peak():
         return 6650.0, "fallback"
 
 
+def fp4_peak():
+    """Dense FP4 tensor-core peak: the measured BF16 GEMM peak (burst) times 4, the ratio of the
+    nominal dense FP4 and BF16 peaks (9 and 2.25 PFLOP/s)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            v = json.load(f).get("bf16_tflops")
+        if v:
+            return round(4.0 * float(v), 1), "measured bf16 x 4"
+    return 4.0 * 1590.0, "fallback bf16 x 4"
+
+
 def ncu_traffic(kernel: str):
     """Per-launch DRAM traffic of `kernel` from the committed ncu summary, or None when the
     kernel's source changed after the capture (the summary stores the source hash)."""
@@ -291,6 +303,48 @@ def run_reference(args, rank, world):
 
 
 # ---- GPU legs ------------------------------------------------------------------------------
+
+def gemm_leg(nv, torch, dev, peak_tflops, m=8192, n=4096, k=4096, reps=20):
+    """The block-scaled FP4 GEMM on a transformer-layer shape (m tokens x k -> n): activations
+    quantized once (Four Over Six, MSE) then nvfp4_gemm, and the variant that quantizes them in
+    its prologue. TFLOP/s = 2 m n k / t against the FP4 dense peak."""
+    gen = torch.Generator(device=dev).manual_seed(7)
+    x = (torch.randn(m, k, device=dev, generator=gen) * torch.exp(torch.randn(k, device=dev, generator=gen))
+         ).to(torch.bfloat16)
+    w = (torch.randn(n, k, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+    wq = nv.quantize_for_gemm(w)
+    ax = nv.amax(x, 1)
+    xq = nv.quantize_for_gemm(x, amax_values=ax)
+    y = torch.empty(m, n, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    s = torch.cuda.current_stream(dev).cuda_stream
+    legs = {
+        "quantize_x": lambda: nv.nvfp4_quantize_gemm(x, m, k, ax, 1, 2, xq[0], xq[1], xq[2], None, s),
+        "gemm": lambda: nv.nvfp4_gemm(xq[0], xq[1], xq[2], wq[0], wq[1], wq[2], m, n, k, y, status, s),
+        "prologue": lambda: nv.nvfp4_gemm_quantize_x(x, ax, 1, 2, wq[0], wq[1], wq[2], m, n, k, y, status, s),
+    }
+    ms = {}
+    for name, fn in legs.items():
+        for _ in range(3):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        b.synchronize()
+        ms[name] = a.elapsed_time(b) / reps
+    flops = 2.0 * m * n * k
+    tf = flops / (ms["gemm"] * 1e-3) / 1e12
+    out = {"shape": [m, n, k], "kernel": "gemm_fp4_kernel (tcgen05.mma.kind::mxf4nvf4.block_scale.block16)",
+           "ms": {k2: round(v, 4) for k2, v in ms.items()}, "tflops": round(tf, 1),
+           "peak_tflops": peak_tflops, "frac": round(tf / peak_tflops, 4),
+           "quantize_then_gemm_tflops": round(flops / ((ms["gemm"] + ms["quantize_x"]) * 1e-3) / 1e12, 1),
+           "prologue_tflops": round(flops / (ms["prologue"] * 1e-3) / 1e12, 1),
+           "status": int(status.item())}
+    del x, w, wq, xq, y
+    return out
+
 
 L2_BYTES = 126 * 2**20
 
@@ -533,6 +587,11 @@ def run_ours(args, rank, world, local):
         per_cfg = per_config_leg(nv, torch, dev, stream, measured_peak()[0],
                                  resident={WORKLOAD: (x_np, (g, r, c))} if args.rows is None else None)
 
+    # ---- the FP4 tensor-core GEMM (N = 1 only) ----
+    gemm = None
+    if world == 1 and not args.no_per_config:
+        gemm = gemm_leg(nv, torch, dev, fp4_peak()[0])
+
     # ---- CPU oracle on a bounded sample (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -577,6 +636,9 @@ def run_ours(args, rank, world, local):
         }
         if per_cfg is not None:
             line["per_config"] = per_cfg
+        if gemm is not None:
+            gemm["peak_kind"] = fp4_peak()[1]
+            line["gemm_fp4"] = gemm
         if cpu is not None:
             line["cpu_baseline"] = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample", "single_thread")}
         print(json.dumps(line), flush=True)
