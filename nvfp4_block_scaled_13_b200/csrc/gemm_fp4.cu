@@ -222,31 +222,43 @@ struct GemmParams {
     int64_t m, n, k;
 };
 
-// Grid (n / 256, m / 128). tmap_a / tmap_b: the codes of x / w as [rows, k/2] byte matrices,
-// boxes of 128 bytes x 128 (A) or 256 (B) rows, 128-byte swizzle (tmap_a unused when QUANT).
+// Persistent: grid = min(tiles, SMs), CTA b takes output tiles b, b + grid, ... in row-major
+// tile order (tm = t / (n / 256), tn = t % (n / 256)). tmap_a / tmap_b: the codes of x / w as
+// [rows, k/2] byte matrices, boxes of 128 bytes x 128 (A) or 256 (B) rows, 128-byte swizzle
+// (tmap_a unused in the prologue variant). Warps: 0 producer lane, 1 MMA lane (and tensor-memory
+// allocation), 2-5 epilogue (tensor-memory lane quarter = warp % 4), 6-11 quantizers (prologue
+// variant). The ring of K slices runs on across tiles, so the next tile's operands stream in
+// while the epilogue drains the accumulator; the MMA lane waits for "accumulator empty" (the
+// four epilogue warps) before a tile's first MMA.
+template <bool QUANT>
+constexpr int gemm_threads() { return QUANT ? 384 : 192; }
+
 template <bool QUANT, bool FOUR, int RULE>
-__global__ void __launch_bounds__(QUANT ? 256 : 128, 1)
+__global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full[kStages], empty[kStages], done;
+    __shared__ __align__(8) uint64_t full[kStages], empty[kStages], acc_full, acc_empty, drain;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile uint32_t stop_sh;
     __shared__ float2 tab[128];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t tn = blockIdx.x, tm = blockIdx.y;
     const int64_t n_ct = p.k / 64;                   // scale tiles per 128 rows
     const int nk = static_cast<int>(p.k / kBK);
+    const int64_t ntn = p.n / kBN, ntiles = (p.m / kBM) * ntn;
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    const uint32_t full0 = smem_u32(&full[0]), empty0 = smem_u32(&empty[0]), done_bar = smem_u32(&done);
+    const uint32_t full0 = smem_u32(&full[0]), empty0 = smem_u32(&empty[0]);
+    const uint32_t accf = smem_u32(&acc_full), acce = smem_u32(&acc_empty), drain_bar = smem_u32(&drain);
 
-    if (warp == 0) tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
-    if (tid == 32) {
+    if (warp == 1) tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
+    if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(full0 + 8 * s, QUANT ? 1 + kQuantWarps : 1);
             mbar_init(empty0 + 8 * s, 1);
         }
-        mbar_init(done_bar, 1);
+        mbar_init(accf, 1);
+        mbar_init(acce, 4);
+        mbar_init(drain_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         stop_sh = 0;
     }
@@ -262,114 +274,150 @@ __global__ void __launch_bounds__(QUANT ? 256 : 128, 1)
     const uint32_t tmem = tmem_base_sh;
 
     if (warp == 0) {
-        if (lane == 0) {   // producer: TMA and bulk copies into the ring
-            for (int ks = 0; ks < nk && !stop_sh; ++ks) {
-                const int s = ks % kStages;
-                const uint32_t u = static_cast<uint32_t>(ks / kStages);
-                if (ks >= kStages && !mbar_wait(empty0 + 8 * s, (u - 1) & 1)) {
-                    stop_sh = 1;
-                    break;
+        if (lane == 0) {   // producer: TMA and bulk copies into the ring, tile after tile
+            int g = 0;
+            for (int64_t t = blockIdx.x; t < ntiles && !stop_sh; t += gridDim.x) {
+                const int64_t tm = t / ntn, tn = t % ntn;
+                for (int ks = 0; ks < nk; ++ks, ++g) {
+                    const int s = g % kStages;
+                    const uint32_t u = static_cast<uint32_t>(g / kStages);
+                    if (g >= kStages && !mbar_wait(empty0 + 8 * s, (u - 1) & 1)) {
+                        stop_sh = 1;
+                        break;
+                    }
+                    const uint32_t fb = full0 + 8 * s, sA = sbase + s * kStageBytes, sB = sA + kABytes;
+                    const uint32_t sSFA = sB + kBBytes, sSFB = sSFA + kSfaBytes;
+                    mbar_expect_tx(fb, (QUANT ? 0u : kABytes + kSfaBytes) + kBBytes + kSfbBytes);
+                    if (!QUANT) {
+                        tma_load_2d(sA, &tmap_a, ks * (kBK / 2), static_cast<int32_t>(tm * kBM), fb);
+                        bulk_load(sSFA, p.x_scales + (tm * n_ct + 4 * ks) * 512, kSfaBytes, fb);
+                    }
+                    tma_load_2d(sB, &tmap_b, ks * (kBK / 2), static_cast<int32_t>(tn * kBN), fb);
+                    bulk_load(sSFB, p.w_scales + (2 * tn * n_ct + 4 * ks) * 512, kSfbBytes / 2, fb);
+                    bulk_load(sSFB + kSfbBytes / 2, p.w_scales + ((2 * tn + 1) * n_ct + 4 * ks) * 512, kSfbBytes / 2,
+                              fb);
                 }
-                const uint32_t fb = full0 + 8 * s, sA = sbase + s * kStageBytes, sB = sA + kABytes;
-                const uint32_t sSFA = sB + kBBytes, sSFB = sSFA + kSfaBytes;
-                mbar_expect_tx(fb, (QUANT ? 0u : kABytes + kSfaBytes) + kBBytes + kSfbBytes);
-                if (!QUANT) {
-                    tma_load_2d(sA, &tmap_a, ks * (kBK / 2), static_cast<int32_t>(tm * kBM), fb);
-                    bulk_load(sSFA, p.x_scales + (tm * n_ct + 4 * ks) * 512, kSfaBytes, fb);
-                }
-                tma_load_2d(sB, &tmap_b, ks * (kBK / 2), static_cast<int32_t>(tn * kBN), fb);
-                bulk_load(sSFB, p.w_scales + (2 * tn * n_ct + 4 * ks) * 512, kSfbBytes / 2, fb);
-                bulk_load(sSFB + kSfbBytes / 2, p.w_scales + ((2 * tn + 1) * n_ct + 4 * ks) * 512, kSfbBytes / 2, fb);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {   // MMA issuer
-            for (int ks = 0; ks < nk && !stop_sh; ++ks) {
-                const int s = ks % kStages;
-                const uint32_t u = static_cast<uint32_t>(ks / kStages);
-                if (!mbar_wait(full0 + 8 * s, u & 1)) {
+            int g = 0, j = 0;
+            for (int64_t t = blockIdx.x; t < ntiles && !stop_sh; t += gridDim.x, ++j) {
+                if (j > 0 && !mbar_wait(acce, (j - 1) & 1)) {   // the epilogue has drained tile j - 1
                     stop_sh = 1;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t sA = sbase + s * kStageBytes, sB = sA + kABytes;
-                const uint32_t sSFA = sB + kBBytes, sSFB = sSFA + kSfaBytes;
-                const uint32_t ca = tmem + kColSfa + 16 * s, cb = tmem + kColSfb + 32 * s;
+                bool ok = true;
+                for (int ks = 0; ks < nk; ++ks, ++g) {
+                    const int s = g % kStages;
+                    const uint32_t u = static_cast<uint32_t>(g / kStages);
+                    if (!mbar_wait(full0 + 8 * s, u & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sA = sbase + s * kStageBytes, sB = sA + kABytes;
+                    const uint32_t sSFA = sB + kBBytes, sSFB = sSFA + kSfaBytes;
+                    const uint32_t ca = tmem + kColSfa + 16 * s, cb = tmem + kColSfb + 32 * s;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    tmem_copy_sf(ca + 4 * j, smem_desc(sSFA + 512 * j, 16, 128));
-                    tmem_copy_sf(cb + 8 * j, smem_desc(sSFB + 512 * j, 16, 128));                   // rows 0..127
-                    tmem_copy_sf(cb + 8 * j + 4, smem_desc(sSFB + kSfbBytes / 2 + 512 * j, 16, 128));   // 128..255
+                    for (int jj = 0; jj < 4; ++jj) {
+                        tmem_copy_sf(ca + 4 * jj, smem_desc(sSFA + 512 * jj, 16, 128));
+                        tmem_copy_sf(cb + 8 * jj, smem_desc(sSFB + 512 * jj, 16, 128));                   // rows 0..127
+                        tmem_copy_sf(cb + 8 * jj + 4, smem_desc(sSFB + kSfbBytes / 2 + 512 * jj, 16, 128));   // 128..255
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj)
+                        mma_fp4(tmem, smem_desc_sw128(sA + 32 * jj), smem_desc_sw128(sB + 32 * jj), kIdesc,
+                                ca + 4 * jj, cb + 8 * jj, (ks | jj) != 0);
+                    mma_commit(empty0 + 8 * s);
                 }
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    mma_fp4(tmem, smem_desc_sw128(sA + 32 * j), smem_desc_sw128(sB + 32 * j), kIdesc, ca + 4 * j,
-                            cb + 8 * j, (ks | j) != 0);
-                mma_commit(empty0 + 8 * s);
-            }
-            mma_commit(done_bar);   // arrives once every MMA issued above has completed
-        }
-    } else if (QUANT) {   // warps 2..7: quantize the stage's activations into the A tile
-        const int q = tid - 64;
-        for (int ks = 0; ks < nk && !stop_sh; ++ks) {
-            const int s = ks % kStages;
-            const uint32_t u = static_cast<uint32_t>(ks / kStages);
-            if (ks >= kStages) {
-                uint32_t ok = 1;
-                if (lane == 0) ok = mbar_wait(empty0 + 8 * s, (u - 1) & 1);
-                if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+                if (!ok) {
                     stop_sh = 1;
                     break;
                 }
+                mma_commit(accf);   // the tile's accumulator is complete once these MMAs are
             }
-            const uint32_t sA = sbase + s * kStageBytes, sSFA = sA + kABytes + kBBytes;
-            // 1024 chunks of 32 elements (two blocks): chunk c = row c / 8, K chunk c % 8
-            for (int c = q; c < 1024; c += 32 * kQuantWarps) {
-                const int r = c >> 3, kc = c & 7;
-                const uint16_t* xs = p.x + (tm * kBM + r) * p.k + ks * kBK + kc * 32;
-                uint32_t w0[8], w1[8], c0lo, c0hi, c1lo, c1hi, s0, s1, h[8];
-                float d;
-                ld32_stream(xs, w0);
-                ld32_stream(xs + 16, w1);
-                quantize_block_regs<FOUR, RULE, false, true>(w0, gc, tab, c0lo, c0hi, s0, d, h);
-                quantize_block_regs<FOUR, RULE, false, true>(w1, gc, tab, c1lo, c1hi, s1, d, h);
-                // 128-byte swizzle: 16-byte chunk kc of row r at r * 128 + (kc ^ (r % 8)) * 16
-                sts16(sA + r * 128 + ((kc ^ (r & 7)) << 4), make_uint4(c0lo, c0hi, c1lo, c1hi));
-                // scale tile of MMA kc / 2: row r, K block j at (r % 32) * 16 + (r / 32) * 4 + j
-                sts16b(sSFA + (kc >> 1) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (kc & 1) * 2,
-                       static_cast<uint16_t>(s0 | (s1 << 8)));
-            }
-            fence_async_smem();   // the stores are read by the tensor core (async proxy)
-            __syncwarp();
-            if (lane == 0) mbar_arrive(full0 + 8 * s);
+            mma_commit(drain_bar);   // arrives when every MMA issued above has completed
+            if (!mbar_wait(drain_bar, 0)) stop_sh = 1;
         }
-    }
-    __syncthreads();   // every role has left its loop
-    if (tid == 0 && !mbar_wait(done_bar, 0)) stop_sh = 1;   // in-flight MMAs, bounded
-    __syncthreads();
-    tc_fence_after();
-    if (!stop_sh) {
-        if (warp < 4) {   // warp w reads tensor-memory lanes (rows) 32w..32w+31
-            const int64_t row = tm * kBM + 32 * warp + lane;
-            float* yr = p.y + row * p.n + tn * kBN;
+    } else if (warp < 6) {   // epilogue: warps 2-5 read tensor-memory lane quarters 2, 3, 0, 1
+        const int q = warp & 3;
+        int j = 0;
+        for (int64_t t = blockIdx.x; t < ntiles && !stop_sh; t += gridDim.x, ++j) {
+            const int64_t tm = t / ntn, tn = t % ntn;
+            uint32_t ok = 1;
+            if (lane == 0) ok = mbar_wait(accf, j & 1);
+            if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+                stop_sh = 1;
+                break;
+            }
+            tc_fence_after();
             const float alpha = (QUANT ? gc.alpha : __ldg(p.x_tscale)) * __ldg(p.w_tscale);
+            float* yr = p.y + (tm * kBM + 32 * q + lane) * p.n + tn * kBN;
 #pragma unroll 1
             for (int c = 0; c < kBN; c += 32) {
                 uint32_t r[32];
-                tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + c, r);
+                tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + c, r);
 #pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4*>(yr + c + j) =
-                        make_float4(__uint_as_float(r[j]) * alpha, __uint_as_float(r[j + 1]) * alpha,
-                                    __uint_as_float(r[j + 2]) * alpha, __uint_as_float(r[j + 3]) * alpha);
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4*>(yr + c + e) =
+                        make_float4(__uint_as_float(r[e]) * alpha, __uint_as_float(r[e + 1]) * alpha,
+                                    __uint_as_float(r[e + 2]) * alpha, __uint_as_float(r[e + 3]) * alpha);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce);
+        }
+    } else if (QUANT) {   // warps 6-11: quantize each slice's activations into the A tile
+        const int qt = tid - 192;
+        int g = 0;
+        for (int64_t t = blockIdx.x; t < ntiles && !stop_sh; t += gridDim.x) {
+            const int64_t tm = t / ntn;
+            bool ok = true;
+            for (int ks = 0; ks < nk; ++ks, ++g) {
+                const int s = g % kStages;
+                const uint32_t u = static_cast<uint32_t>(g / kStages);
+                if (g >= kStages) {
+                    uint32_t w = 1;
+                    if (lane == 0) w = mbar_wait(empty0 + 8 * s, (u - 1) & 1);
+                    if (!__shfl_sync(0xFFFFFFFFu, w, 0)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                const uint32_t sA = sbase + s * kStageBytes, sSFA = sA + kABytes + kBBytes;
+                // 1024 chunks of 32 elements (two blocks): chunk c = row c / 8, K chunk c % 8
+                for (int c = qt; c < 1024; c += 32 * kQuantWarps) {
+                    const int r = c >> 3, kc = c & 7;
+                    const uint16_t* xs = p.x + (tm * kBM + r) * p.k + ks * kBK + kc * 32;
+                    uint32_t w0[8], w1[8], c0lo, c0hi, c1lo, c1hi, s0, s1, h[8];
+                    float d;
+                    ld32_stream(xs, w0);
+                    ld32_stream(xs + 16, w1);
+                    quantize_block_regs<FOUR, RULE, false, true>(w0, gc, tab, c0lo, c0hi, s0, d, h);
+                    quantize_block_regs<FOUR, RULE, false, true>(w1, gc, tab, c1lo, c1hi, s1, d, h);
+                    // 128-byte swizzle: 16-byte chunk kc of row r at r * 128 + (kc ^ (r % 8)) * 16
+                    sts16(sA + r * 128 + ((kc ^ (r & 7)) << 4), make_uint4(c0lo, c0hi, c1lo, c1hi));
+                    // scale tile of MMA kc / 2: row r, K block j at (r % 32) * 16 + (r / 32) * 4 + j
+                    sts16b(sSFA + (kc >> 1) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (kc & 1) * 2,
+                           static_cast<uint16_t>(s0 | (s1 << 8)));
+                }
+                fence_async_smem();   // the stores are read by the tensor core (async proxy)
+                __syncwarp();
+                if (lane == 0) mbar_arrive(full0 + 8 * s);
+            }
+            if (!ok) {
+                stop_sh = 1;
+                break;
             }
         }
-    } else if (tid == 0 && p.status != nullptr) {
-        atomicOr(p.status, NVFP4_GEMM_TIMEOUT);
     }
     tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+    __syncthreads();   // every role has left its loop; the MMA lane has drained the tensor core
+    if (stop_sh && tid == 0 && p.status != nullptr) atomicOr(p.status, NVFP4_GEMM_TIMEOUT);
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
 // ---- host side -----------------------------------------------------------------------------------
@@ -410,8 +458,12 @@ nvfp4_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const Gem
     // per device, so set on every launch (cheap)
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem) != cudaSuccess)
         return NVFP4_ERR_CUDA;
-    const dim3 grid(static_cast<unsigned>(p.n / kBN), static_cast<unsigned>(p.m / kBM));
-    kernel<<<grid, QUANT ? 256 : 128, kDynSmem, stream>>>(ma, mb, p);
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    const int64_t tiles = (p.m / kBM) * (p.n / kBN);
+    const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);   // one CTA per SM
+    kernel<<<grid, gemm_threads<QUANT>(), kDynSmem, stream>>>(ma, mb, p);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
