@@ -209,37 +209,55 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p)
 
 // ---- dequantize ------------------------------------------------------------------------------
 
+// Thread i dequantizes blocks 2i and 2i + 1 per step (grid-strided over pairs): two 8-byte code
+// loads and two scale bytes, prefetched one step ahead, and 64 contiguous bytes of BF16 out, so
+// a warp reads 512 contiguous bytes of codes and writes 2 KiB. The two blocks of a pair may sit
+// in different groups; each looks its tensor scale up when it passes the cached group end.
 __global__ void __launch_bounds__(kThreads, 4) dequantize_kernel(const DequantParams p) {
+    const int64_t npairs = (p.nblocks + 1) >> 1;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-    int64_t b = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
+    int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
     int64_t g_end = 0;
     float alpha = 0.0f;
-    uint32_t nlo = 0, nhi = 0, ns = 0;
-    if (b < p.nblocks) {
-        ld8_stream(p.codes + b * 8, nlo, nhi);
-        ns = ld1_stream(p.scales + b);
+    uint32_t n0lo = 0, n0hi = 0, n1lo = 0, n1hi = 0, ns0 = 0, ns1 = 0;
+    if (i < npairs) {
+        ld8_stream(p.codes + i * 16, n0lo, n0hi);
+        ns0 = ld1_stream(p.scales + 2 * i);
+        if (2 * i + 1 < p.nblocks) {
+            ld8_stream(p.codes + i * 16 + 8, n1lo, n1hi);
+            ns1 = ld1_stream(p.scales + 2 * i + 1);
+        }
     }
-    for (; b < p.nblocks; b += stride) {
-        const uint32_t clo = nlo, chi = nhi, s = ns;
-        const int64_t bn = b + stride;
-        if (bn < p.nblocks) {
-            ld8_stream(p.codes + bn * 8, nlo, nhi);
-            ns = ld1_stream(p.scales + bn);
+    for (; i < npairs; i += stride) {
+        const uint32_t c[2][2] = {{n0lo, n0hi}, {n1lo, n1hi}}, sc[2] = {ns0, ns1};
+        const int64_t in = i + stride;
+        if (in < npairs) {
+            ld8_stream(p.codes + in * 16, n0lo, n0hi);
+            ns0 = ld1_stream(p.scales + 2 * in);
+            if (2 * in + 1 < p.nblocks) {
+                ld8_stream(p.codes + in * 16 + 8, n1lo, n1hi);
+                ns1 = ld1_stream(p.scales + 2 * in + 1);
+            }
         }
-        if (b >= g_end) {
-            const int64_t g = p.gdiv(b);
-            g_end = g * p.gdiv.bpg + p.gdiv.bpg;
-            alpha = __ldg(p.tscale + g);
-        }
-        const float d = __fmul_rn(e4m3x2_to_float2(s).x, alpha);
-        const float2 dd = make_float2(d, d);
-        uint32_t h[8];
-        e2m1x8_to_f16x2(clo, h[0], h[1], h[2], h[3]);
-        e2m1x8_to_f16x2(chi, h[4], h[5], h[6], h[7]);
-        uint32_t out[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) out[j] = bf16x2(mul2(f16x2_to_float2(h[j]), dd));
-        st32(p.y + b * 16, out);
+        for (int k = 0; k < 2; ++k) {
+            const int64_t b = 2 * i + k;
+            if (b >= p.nblocks) break;
+            if (b >= g_end) {
+                const int64_t g = p.gdiv(b);
+                g_end = g * p.gdiv.bpg + p.gdiv.bpg;
+                alpha = __ldg(p.tscale + g);
+            }
+            const float d = __fmul_rn(e4m3x2_to_float2(sc[k]).x, alpha);
+            const float2 dd = make_float2(d, d);
+            uint32_t h[8];
+            e2m1x8_to_f16x2(c[k][0], h[0], h[1], h[2], h[3]);
+            e2m1x8_to_f16x2(c[k][1], h[4], h[5], h[6], h[7]);
+            uint32_t out[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) out[j] = bf16x2(mul2(f16x2_to_float2(h[j]), dd));
+            st32(p.y + b * 16, out);
+        }
     }
 }
 

@@ -281,7 +281,7 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const
     p.nblocks = n / 16;
     p.groups = groups;
     p.gdiv = make_gdiv(groups, rows * cols / 16, p.nblocks);
-    const unsigned grid = grid_for(nvfp4::dequantize_kernel, p.nblocks);
+    const unsigned grid = grid_for(nvfp4::dequantize_kernel, (p.nblocks + 1) / 2);   // one pair per thread
     nvfp4::dequantize_kernel<<<grid, kThreads, 0, stream>>>(p);
     return launch_status();
 }
