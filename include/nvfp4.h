@@ -1,6 +1,8 @@
 /*
  * nvfp4.h — C ABI of libnvfp4.so: BF16 -> NVFP4 block-scaled quantization on NVIDIA B200
- * (sm_100a), with standard "scale-6" blocks and Four Over Six adaptive block scaling.
+ * (sm_100a), with standard "scale-6" blocks and Four Over Six adaptive block scaling; the
+ * block-scaled FP4 GEMM on the tensor cores that consumes it (optionally quantizing the
+ * activations inside its prologue); and the distillation loss of a QAD student.
  *
  * Sources (web pages, cited by title and section):
  *   [FOS] "Four Over Six: More Accurate NVFP4 Quantization with Adaptive Block Scaling"
@@ -10,6 +12,8 @@
  *         (gist.science explainer), technical summary §3.3: NVFP4 blocks of 16 values.
  *   [N35] "NVIDIA、「Nemotron 3.5 Lightning」のNVFP4量子化手法を公開" (news article), two-stage
  *         QAD section: the student's forward pass runs through simulated quantization.
+ *   [MO]  "NVIDIA Model Optimizerを用いたNemotron 3.5 Lightning NVFP4とQADの開発" (blog), NVFP4
+ *         and QAD sections.
  *
  * The number format. A tensor x of BF16 values, viewed as [groups, rows, cols] row-major, is
  * cut into blocks of 16 consecutive elements along the last dimension ([QAD] §3.3). Each
@@ -39,8 +43,9 @@
  *
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller. The library allocates no
- *     memory, keeps no state between calls and never synchronizes the host: work is enqueued
- *     on `stream` (0 = the legacy default stream) and completes in stream order.
+ *     memory, keeps no state between calls besides cached device attributes, and never
+ *     synchronizes the host: work is enqueued on `stream` (0 = the legacy default stream) and
+ *     completes in stream order.
  *   - Shapes: groups >= 1, rows >= 0, cols >= 0 with cols % 16 == 0. An empty tensor
  *     (rows == 0 or cols == 0) is valid; each function states what it writes for one.
  *   - Alignment: BF16 tensors (x, y) 32 bytes, codes 8 bytes, choice/amax/tscale 4 bytes.
@@ -49,7 +54,9 @@
  *     give unspecified outputs. Output buffers must not overlap inputs or each other.
  *   - Errors: argument errors are detected on the host and returned before anything is
  *     enqueued (no output is touched). A launch failure returns NVFP4_ERR_CUDA. Kernels
- *     contain no device-side assert, trap or wait.
+ *     contain no device-side assert or trap. The only waits are the GEMM's mbarrier waits on
+ *     its own copies and tensor-core work; each is bounded (about two seconds) and reports a
+ *     timeout through the GEMM's status word.
  *   - Buffers must live on the device that is current for the calling thread.
  */
 #ifndef NVFP4_H
