@@ -123,20 +123,20 @@ __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kerne
     const uint32_t warps = gridDim.x * (kThreads / 32);
     const uint32_t warp0 = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
     for (int64_t g = blockIdx.y; g < p.groups; g += gridDim.y) {
+        const int64_t base = g * static_cast<int64_t>(bpg);
+        const uint16_t* xg = p.x + base * 16;
+        uint32_t tile = warp0;
+        uint32_t a0[8], a1[8];
+        if (tile < ntiles) load_tile(xg, tile, lane, bpg, a0, a1);   // in flight while the table is built
         const GroupCtx gc = make_group<FOUR>(__ldg(p.amax + g), kSixM);
         __syncthreads();                       // the previous group's table is no longer read
         if (threadIdx.x < 128) tab[threadIdx.x] = scale_entry(threadIdx.x == 127 ? 126u : threadIdx.x, gc.alpha);
         if (!FQ && blockIdx.x == 0 && threadIdx.x == 0) p.tscale[g] = gc.alpha;
         __syncthreads();
-        const int64_t base = g * static_cast<int64_t>(bpg);
-        const uint16_t* xg = p.x + base * 16;
         uint8_t* cg = FQ ? nullptr : p.codes + base * 8;
         uint8_t* sg = FQ ? nullptr : p.scales + base;
         uint16_t* yg = FQ ? p.y + base * 16 : nullptr;
         uint32_t* chw = reinterpret_cast<uint32_t*>(p.choice) + (base >> 5);   // base is a multiple of 32
-        uint32_t tile = warp0;
-        uint32_t a0[8], a1[8];
-        if (tile < ntiles) load_tile(xg, tile, lane, bpg, a0, a1);
         if constexpr (!FOUR) {   // one prefetch buffer: two would not fit the 64-register budget
             for (; tile < ntiles; tile += warps) {
                 uint32_t b0[8], b1[8];

@@ -130,3 +130,46 @@ def test_side_stream_and_status_word(gpu):
     s.synchronize()
     assert status.item() == 0
     assert torch.equal(y.view(torch.int32), y_ref.view(torch.int32))
+
+
+def test_more_tiles_than_ctas(gpu):
+    """2048 x 4096 x 512: 256 output tiles on one CTA per SM, so CTAs run one or two tiles and
+    hand the accumulator over between them; every output against the exact product."""
+    m, n, k = 2048, 4096, 512
+    x, w = operands(m, n, k, seed=17)
+    xd, wd = device_bf16(x, m, k), device_bf16(w, n, k)
+    xq, wq = nv.quantize_for_gemm(xd), nv.quantize_for_gemm(wd)
+    y = nv.gemm(xq, wq)
+    y2 = nv.gemm_quantize_x(xd, wq)
+    assert torch.equal(y.view(torch.int32), y2.view(torch.int32))
+    xc, xs, xt = oracle_quant(x, m, k, "four_over_six", "mse")
+    wc, ws, wt = oracle_quant(w, n, k, "four_over_six", "mse")
+    want = O.gemm_nvfp4(xc, xs, xt, wc, ws, wt, m, n, k)
+    s = O.gemm_nvfp4(magnitude(xc), xs, xt, magnitude(wc), ws, wt, m, n, k)
+    err = np.abs(y.cpu().numpy().astype(np.float64) - want)
+    assert np.all(err <= (k / 64 + 4) * 2.0 ** -22 * s + 1e-30)
+
+
+@pytest.mark.slow
+def test_bench_shape_sampled(gpu):
+    """The bench's GEMM shape, 8192 x 4096 x 4096 (2048 tiles, about 14 per CTA): 512 sampled
+    outputs (whole rows' worth of tiles included) against the exact product of the oracle's
+    operands."""
+    m, n, k = 8192, 4096, 4096
+    rng = np.random.default_rng(8)
+    x, w = operands(m, n, k, seed=23)
+    xd, wd = device_bf16(x, m, k), device_bf16(w, n, k)
+    xq, wq = nv.quantize_for_gemm(xd), nv.quantize_for_gemm(wd)
+    y = nv.gemm(xq, wq).cpu().numpy().astype(np.float64)
+    xc, xs, xt = oracle_quant(x, m, k, "four_over_six", "mse")
+    wc, ws, wt = oracle_quant(w, n, k, "four_over_six", "mse")
+    assert np.array_equal(xq[0].cpu().numpy().ravel(), xc) and np.array_equal(wq[0].cpu().numpy().ravel(), wc)
+    rows = np.concatenate([rng.integers(0, m, 14), [0, m - 1]])
+    cols = np.concatenate([rng.integers(0, n, 30), [0, n - 1]])
+    xr, xsr = xc.reshape(m, k // 2)[rows], xs.reshape(m, k // 16)[rows]
+    wr, wsr = wc.reshape(n, k // 2)[cols], ws.reshape(n, k // 16)[cols]
+    want = O.gemm_nvfp4(xr, xsr, xt, wr, wsr, wt, len(rows), len(cols), k)
+    s = O.gemm_nvfp4(magnitude(xr), xsr, xt, magnitude(wr), wsr, wt, len(rows), len(cols), k)
+    got = y[np.ix_(rows, cols)]
+    assert np.all(np.abs(got - want) <= (k / 64 + 4) * 2.0 ** -22 * s + 1e-30)
+    assert np.all(np.isfinite(y))
