@@ -75,13 +75,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait for the mbarrier phase with the given parity to complete.
+// Bounded wait for the mbarrier phase with the given parity to complete (the clock is read
+// once per 64 polls, so that the common case costs one try_wait).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
         if (clock64() - t0 > kWaitCycles) return false;
     }
-    return true;
 }
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -182,18 +186,36 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
                  : "memory");
 }
 
-// 32 lanes x 32 consecutive 32-bit columns of tensor memory -> 32 registers per thread.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+// 32 lanes x 64 consecutive 32-bit columns of tensor memory -> 64 registers per thread; the
+// registers are valid after tmem_wait_ld().
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
           "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
         : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 8 consecutive FP32 outputs (a 32-byte sector), each accumulator word times alpha.
+__device__ __forceinline__ void st_v8f(float* dst, const uint32_t* r, float alpha) {
+    asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst),
+                 "f"(__uint_as_float(r[0]) * alpha), "f"(__uint_as_float(r[1]) * alpha),
+                 "f"(__uint_as_float(r[2]) * alpha), "f"(__uint_as_float(r[3]) * alpha),
+                 "f"(__uint_as_float(r[4]) * alpha), "f"(__uint_as_float(r[5]) * alpha),
+                 "f"(__uint_as_float(r[6]) * alpha), "f"(__uint_as_float(r[7]) * alpha)
+                 : "memory");
 }
 
 __device__ __forceinline__ void sts16(uint32_t addr, uint4 v) {
@@ -300,44 +322,56 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {   // MMA issuer
-            int g = 0, j = 0;
-            for (int64_t t = blockIdx.x; t < ntiles && !stop_sh; t += gridDim.x, ++j) {
-                if (j > 0 && !mbar_wait(acce, (j - 1) & 1)) {   // the epilogue has drained tile j - 1
-                    stop_sh = 1;
-                    break;
-                }
-                tc_fence_after();
-                bool ok = true;
-                for (int ks = 0; ks < nk; ++ks, ++g) {
-                    const int s = g % kStages;
-                    const uint32_t u = static_cast<uint32_t>(g / kStages);
-                    if (!mbar_wait(full0 + 8 * s, u & 1)) {
+        if (lane == 0) {   // MMA issuer: one thread issues every tcgen05 instruction, so its per-slice
+                           // work is kept to a few instructions: the ring slots are unrolled and their
+                           // descriptors and tensor-memory addresses are immediates off per-slot bases
+            const int64_t my_tiles = (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
+            const int64_t total = my_tiles * nk;
+            const uint64_t dA0 = smem_desc_sw128(sbase), dB0 = smem_desc_sw128(sbase + kABytes);
+            const uint64_t dSA0 = smem_desc(sbase + kABytes + kBBytes, 16, 128);
+            const uint64_t dSB0 = smem_desc(sbase + kABytes + kBBytes + kSfaBytes, 16, 128);
+            constexpr uint64_t kSlot = kStageBytes >> 4;   // descriptor start-address units per slot
+            int64_t gg = 0;
+            int ks = 0, tile_j = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            while (gg < total && ok) {
+#pragma unroll
+                for (int s = 0; s < kStages; ++s) {
+                    if (gg >= total) break;
+                    if (ks == 0 && tile_j > 0) {   // the epilogue has drained tile tile_j - 1
+                        if (!mbar_wait(acce, static_cast<uint32_t>(tile_j - 1) & 1)) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (!mbar_wait(full0 + 8 * s, phase)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sA = sbase + s * kStageBytes, sB = sA + kABytes;
-                    const uint32_t sSFA = sB + kBBytes, sSFB = sSFA + kSfaBytes;
                     const uint32_t ca = tmem + kColSfa + 16 * s, cb = tmem + kColSfb + 32 * s;
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
-                        tmem_copy_sf(ca + 4 * jj, smem_desc(sSFA + 512 * jj, 16, 128));
-                        tmem_copy_sf(cb + 8 * jj, smem_desc(sSFB + 512 * jj, 16, 128));                   // rows 0..127
-                        tmem_copy_sf(cb + 8 * jj + 4, smem_desc(sSFB + kSfbBytes / 2 + 512 * jj, 16, 128));   // 128..255
+                        tmem_copy_sf(ca + 4 * jj, dSA0 + s * kSlot + 32 * jj);
+                        tmem_copy_sf(cb + 8 * jj, dSB0 + s * kSlot + 32 * jj);                 // B rows 0..127
+                        tmem_copy_sf(cb + 8 * jj + 4, dSB0 + s * kSlot + 128 + 32 * jj);       // 128..255
                     }
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj)
-                        mma_fp4(tmem, smem_desc_sw128(sA + 32 * jj), smem_desc_sw128(sB + 32 * jj), kIdesc,
-                                ca + 4 * jj, cb + 8 * jj, (ks | jj) != 0);
+                        mma_fp4(tmem, dA0 + s * kSlot + 2 * jj, dB0 + s * kSlot + 2 * jj, kIdesc, ca + 4 * jj,
+                                cb + 8 * jj, (ks | jj) != 0);
                     mma_commit(empty0 + 8 * s);
+                    ++gg;
+                    if (++ks == nk) {
+                        ks = 0;
+                        ++tile_j;
+                        mma_commit(accf);   // the tile's accumulator is complete once these MMAs are
+                    }
                 }
-                if (!ok) {
-                    stop_sh = 1;
-                    break;
-                }
-                mma_commit(accf);   // the tile's accumulator is complete once these MMAs are
+                phase ^= 1;
             }
+            if (!ok) stop_sh = 1;
             mma_commit(drain_bar);   // arrives when every MMA issued above has completed
             if (!mbar_wait(drain_bar, 0)) stop_sh = 1;
         }
@@ -355,19 +389,29 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
             tc_fence_after();
             const float alpha = (QUANT ? gc.alpha : __ldg(p.x_tscale)) * __ldg(p.w_tscale);
             float* yr = p.y + (tm * kBM + 32 * q + lane) * p.n + tn * kBN;
-#pragma unroll 1
-            for (int c = 0; c < kBN; c += 32) {
-                uint32_t r[32];
-                tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + c, r);
+            const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16);
+            // four chunks of 64 columns: the next chunk's load is in flight while this one is
+            // stored, and the accumulator is released as soon as the last load has landed
+            uint32_t r0[64], r1[64];
+            tmem_ld64(trow, r0);
+            tmem_wait_ld();
+            tmem_ld64(trow + 64, r1);
 #pragma unroll
-                for (int e = 0; e < 32; e += 4)
-                    *reinterpret_cast<float4*>(yr + c + e) =
-                        make_float4(__uint_as_float(r[e]) * alpha, __uint_as_float(r[e + 1]) * alpha,
-                                    __uint_as_float(r[e + 2]) * alpha, __uint_as_float(r[e + 3]) * alpha);
-            }
+            for (int e = 0; e < 64; e += 8) st_v8f(yr + e, r0 + e, alpha);   // whole 32-byte sectors
+            tmem_wait_ld();
+            tmem_ld64(trow + 128, r0);
+#pragma unroll
+            for (int e = 0; e < 64; e += 8) st_v8f(yr + 64 + e, r1 + e, alpha);
+            tmem_wait_ld();
+            tmem_ld64(trow + 192, r1);
+#pragma unroll
+            for (int e = 0; e < 64; e += 8) st_v8f(yr + 128 + e, r0 + e, alpha);
+            tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(acce);
+#pragma unroll
+            for (int e = 0; e < 64; e += 8) st_v8f(yr + 192 + e, r1 + e, alpha);
         }
     } else if (QUANT) {   // warps 6-11: quantize each slice's activations into the A tile
         const int qt = tid - 192;
@@ -490,7 +534,7 @@ extern "C" nvfp4_status nvfp4_gemm(const uint8_t* x_codes, const uint8_t* x_scal
     if (m == 0 || n == 0) return NVFP4_OK;
     if (!x_codes || !x_scales || !x_tscale || !w_codes || !w_scales || !w_tscale || !y) return NVFP4_ERR_NULL;
     if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
-        !aligned16(y) || !aligned4(x_tscale) || !aligned4(w_tscale) || !aligned4(status))
+        (reinterpret_cast<uintptr_t>(y) & 31u) || !aligned4(x_tscale) || !aligned4(w_tscale) || !aligned4(status))
         return NVFP4_ERR_ALIGN;
     if (k == 0) return NVFP4_ERR_SHAPE;
     CUtensorMap ma, mb;
@@ -518,7 +562,8 @@ extern "C" nvfp4_status nvfp4_gemm_quantize_x(const uint16_t* x, const float* x_
     if (rule != NVFP4_RULE_MAXERR && rule != NVFP4_RULE_MAE && rule != NVFP4_RULE_MSE) return NVFP4_ERR_RULE;
     if (m == 0 || n == 0) return NVFP4_OK;
     if (!x || !x_amax || !w_codes || !w_scales || !w_tscale || !y) return NVFP4_ERR_NULL;
-    if ((reinterpret_cast<uintptr_t>(x) & 31u) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y) ||
+    if ((reinterpret_cast<uintptr_t>(x) & 31u) || !aligned16(w_codes) || !aligned16(w_scales) ||
+        (reinterpret_cast<uintptr_t>(y) & 31u) ||
         !aligned4(x_amax) || !aligned4(w_tscale) || !aligned4(status))
         return NVFP4_ERR_ALIGN;
     if (k == 0) return NVFP4_ERR_SHAPE;

@@ -96,6 +96,7 @@ A = 1 << 20          # 32-byte aligned
     (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 128, 256, 256, None, None, None), 1),
     (lambda L: L.nvfp4_gemm(A + 8, A, A, A, A, A, 128, 256, 256, A, None, None), 3),
     (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 128, 256, 256, A, A + 2, None), 3),
+    (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 128, 256, 256, A + 16, None, None), 3),
     (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 0, 256, 256, None, None, None), 0),
     # nvfp4_gemm_quantize_x(x, amax, mode, rule, wc, ws, wt, m, n, k, y, status, stream)
     (lambda L: L.nvfp4_gemm_quantize_x(A, A, 2, 2, A, A, A, 128, 256, 256, A, None, None), 4),
