@@ -196,7 +196,7 @@ NVFP4_API nvfp4_status nvfp4_quantize_gemm(const uint16_t* x, int64_t rows, int6
  *   w_codes [n, k/2], w_scales tiled, w_tscale [1] alpha_w      (in, device)
  *   y       [m, n] FP32                                          (out, device)
  *   status  nullable device word; NVFP4_GEMM_TIMEOUT is or-ed in on a timed-out wait (in/out)
- * m must be a multiple of 128, n and k multiples of 256 (else NVFP4_ERR_SHAPE); codes and
+ * m >= 0 is any row count, n a multiple of 128 and k of 256 (else NVFP4_ERR_SHAPE); codes and
  * scales 16-byte aligned, y 32-byte aligned; the tensor-map encoder of the driver must be available (else
  * NVFP4_ERR_CUDA). The accumulation is FP32 inside the tensor core, so y agrees
  * with the exact product to within FP32 accumulation error, not bit for bit. */

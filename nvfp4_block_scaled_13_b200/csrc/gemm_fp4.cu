@@ -267,7 +267,10 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t n_ct = p.k / 64;                   // scale tiles per 128 rows
     const int nk = static_cast<int>(p.k / kBK);
-    const int64_t ntn = p.n / kBN, ntiles = (p.m / kBM) * ntn;
+    // ragged edges: the last row tile may hold fewer than 128 rows of A (TMA fills the rest
+    // with zeros and the epilogue stores only rows below m), and n a multiple of 128 may end
+    // in a half tile (its second 128 rows of B are zeros and its columns are not stored)
+    const int64_t ntn = (p.n + kBN - 1) / kBN, ntiles = ((p.m + kBM - 1) / kBM) * ntn;
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t full0 = smem_u32(&full[0]), empty0 = smem_u32(&empty[0]);
     const uint32_t accf = smem_u32(&acc_full), acce = smem_u32(&acc_empty), drain_bar = smem_u32(&drain);
@@ -309,15 +312,17 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
                     }
                     const uint32_t fb = full0 + 8 * s, sA = sbase + s * kStageBytes, sB = sA + kABytes;
                     const uint32_t sSFA = sB + kBBytes, sSFB = sSFA + kSfaBytes;
-                    mbar_expect_tx(fb, (QUANT ? 0u : kABytes + kSfaBytes) + kBBytes + kSfbBytes);
+                    const bool b_hi = (2 * tn + 1) * 128 < p.n;   // the tile's second 128 rows of B exist
+                    mbar_expect_tx(fb, (QUANT ? 0u : kABytes + kSfaBytes) + kBBytes + (b_hi ? kSfbBytes : kSfbBytes / 2));
                     if (!QUANT) {
                         tma_load_2d(sA, &tmap_a, ks * (kBK / 2), static_cast<int32_t>(tm * kBM), fb);
                         bulk_load(sSFA, p.x_scales + (tm * n_ct + 4 * ks) * 512, kSfaBytes, fb);
                     }
                     tma_load_2d(sB, &tmap_b, ks * (kBK / 2), static_cast<int32_t>(tn * kBN), fb);
                     bulk_load(sSFB, p.w_scales + (2 * tn * n_ct + 4 * ks) * 512, kSfbBytes / 2, fb);
-                    bulk_load(sSFB + kSfbBytes / 2, p.w_scales + ((2 * tn + 1) * n_ct + 4 * ks) * 512, kSfbBytes / 2,
-                              fb);
+                    if (b_hi)
+                        bulk_load(sSFB + kSfbBytes / 2, p.w_scales + ((2 * tn + 1) * n_ct + 4 * ks) * 512,
+                                  kSfbBytes / 2, fb);
                 }
             }
         }
@@ -388,7 +393,9 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
             }
             tc_fence_after();
             const float alpha = (QUANT ? gc.alpha : __ldg(p.x_tscale)) * __ldg(p.w_tscale);
-            float* yr = p.y + (tm * kBM + 32 * q + lane) * p.n + tn * kBN;
+            const int64_t row = tm * kBM + 32 * q + lane;
+            const bool row_ok = row < p.m, full_n = tn * kBN + kBN <= p.n;
+            float* yr = p.y + (row_ok ? row : 0) * p.n + tn * kBN;
             const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16);
             // four chunks of 64 columns: the next chunk's load is in flight while this one is
             // stored, and the accumulator is released as soon as the last load has landed
@@ -396,22 +403,30 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
             tmem_ld64(trow, r0);
             tmem_wait_ld();
             tmem_ld64(trow + 64, r1);
+            if (row_ok) {
 #pragma unroll
-            for (int e = 0; e < 64; e += 8) st_v8f(yr + e, r0 + e, alpha);   // whole 32-byte sectors
+                for (int e = 0; e < 64; e += 8) st_v8f(yr + e, r0 + e, alpha);   // whole 32-byte sectors
+            }
             tmem_wait_ld();
             tmem_ld64(trow + 128, r0);
+            if (row_ok) {
 #pragma unroll
-            for (int e = 0; e < 64; e += 8) st_v8f(yr + 64 + e, r1 + e, alpha);
+                for (int e = 0; e < 64; e += 8) st_v8f(yr + 64 + e, r1 + e, alpha);
+            }
             tmem_wait_ld();
             tmem_ld64(trow + 192, r1);
+            if (row_ok && full_n) {
 #pragma unroll
-            for (int e = 0; e < 64; e += 8) st_v8f(yr + 128 + e, r0 + e, alpha);
+                for (int e = 0; e < 64; e += 8) st_v8f(yr + 128 + e, r0 + e, alpha);
+            }
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(acce);
+            if (row_ok && full_n) {
 #pragma unroll
-            for (int e = 0; e < 64; e += 8) st_v8f(yr + 192 + e, r1 + e, alpha);
+                for (int e = 0; e < 64; e += 8) st_v8f(yr + 192 + e, r1 + e, alpha);
+            }
         }
     } else if (QUANT) {   // warps 6-11: quantize each slice's activations into the A tile
         const int qt = tid - 192;
@@ -434,11 +449,14 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
                 // 1024 chunks of 32 elements (two blocks): chunk c = row c / 8, K chunk c % 8
                 for (int c = qt; c < 1024; c += 32 * kQuantWarps) {
                     const int r = c >> 3, kc = c & 7;
-                    const uint16_t* xs = p.x + (tm * kBM + r) * p.k + ks * kBK + kc * 32;
-                    uint32_t w0[8], w1[8], c0lo, c0hi, c1lo, c1hi, s0, s1, h[8];
+                    const int64_t row = tm * kBM + r;
+                    uint32_t w0[8] = {}, w1[8] = {}, c0lo, c0hi, c1lo, c1hi, s0, s1, h[8];
                     float d;
-                    ld32_stream(xs, w0);
-                    ld32_stream(xs + 16, w1);
+                    if (row < p.m) {   // rows past m quantize as zeros (codes 0, scale 0)
+                        const uint16_t* xs = p.x + row * p.k + ks * kBK + kc * 32;
+                        ld32_stream(xs, w0);
+                        ld32_stream(xs + 16, w1);
+                    }
                     quantize_block_regs<FOUR, RULE, false, true>(w0, gc, tab, c0lo, c0hi, s0, d, h);
                     quantize_block_regs<FOUR, RULE, false, true>(w1, gc, tab, c1lo, c1hi, s1, d, h);
                     // 128-byte swizzle: 16-byte chunk kc of row r at r * 128 + (kc ^ (r % 8)) * 16
@@ -505,7 +523,7 @@ nvfp4_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const Gem
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return NVFP4_ERR_CUDA;
-    const int64_t tiles = (p.m / kBM) * (p.n / kBN);
+    const int64_t tiles = ((p.m + kBM - 1) / kBM) * ((p.n + kBN - 1) / kBN);
     const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);   // one CTA per SM
     kernel<<<grid, gemm_threads<QUANT>(), kDynSmem, stream>>>(ma, mb, p);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
@@ -516,10 +534,8 @@ bool aligned4(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 3u) == 0
 
 nvfp4_status check_gemm_shape(int64_t m, int64_t n, int64_t k) {
     if (m < 0 || n < 0 || k < 0) return NVFP4_ERR_SHAPE;
-    if (m % kBM || n % kBN || k % kBK) return NVFP4_ERR_SHAPE;
-    if (m / kBM > 65535 || n / kBN > 65535 || k > (int64_t(1) << 30) || m > (int64_t(1) << 31) ||
-        n > (int64_t(1) << 31))
-        return NVFP4_ERR_SHAPE;
+    if (n % 128 || k % kBK) return NVFP4_ERR_SHAPE;
+    if (k > (int64_t(1) << 30) || m > (int64_t(1) << 31) || n > (int64_t(1) << 31)) return NVFP4_ERR_SHAPE;
     return NVFP4_OK;
 }
 

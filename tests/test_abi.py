@@ -88,9 +88,9 @@ A = 1 << 20          # 32-byte aligned
     (lambda L: L.nvfp4_qad_kl(A + 1, A, 4, 8, 1.0, 1.0, A, None, None), 3),
     (lambda L: L.nvfp4_qad_kl(A, A, 4, 8, 1.0, 1.0, A + 2, None, None), 3),
     # nvfp4_gemm(xc, xs, xt, wc, ws, wt, m, n, k, y, status, stream)
-    (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 100, 256, 256, A, None, None), 2),
     (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 128, 256, 200, A, None, None), 2),
-    (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 128, 128, 256, A, None, None), 2),
+    (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 128, 192, 256, A, None, None), 2),
+    (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, -1, 256, 256, A, None, None), 2),
     (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 128, 256, 0, A, None, None), 2),
     (lambda L: L.nvfp4_gemm(None, A, A, A, A, A, 128, 256, 256, A, None, None), 1),
     (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 128, 256, 256, None, None, None), 1),
@@ -102,6 +102,7 @@ A = 1 << 20          # 32-byte aligned
     (lambda L: L.nvfp4_gemm_quantize_x(A, A, 2, 2, A, A, A, 128, 256, 256, A, None, None), 4),
     (lambda L: L.nvfp4_gemm_quantize_x(A, A, 1, 3, A, A, A, 128, 256, 256, A, None, None), 5),
     (lambda L: L.nvfp4_gemm_quantize_x(A, A, 1, 2, A, A, A, 128, 64, 256, A, None, None), 2),
+    (lambda L: L.nvfp4_gemm_quantize_x(A, A, 1, 2, A, A, A, 100, 128, 320, A, None, None), 2),
     (lambda L: L.nvfp4_gemm_quantize_x(None, A, 1, 2, A, A, A, 128, 256, 256, A, None, None), 1),
     (lambda L: L.nvfp4_gemm_quantize_x(A, None, 1, 2, A, A, A, 128, 256, 256, A, None, None), 1),
     (lambda L: L.nvfp4_gemm_quantize_x(A + 16, A, 1, 2, A, A, A, 128, 256, 256, A, None, None), 3),

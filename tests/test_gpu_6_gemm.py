@@ -173,3 +173,31 @@ def test_bench_shape_sampled(gpu):
     got = y[np.ix_(rows, cols)]
     assert np.all(np.abs(got - want) <= (k / 64 + 4) * 2.0 ** -22 * s + 1e-30)
     assert np.all(np.isfinite(y))
+
+
+RAGGED = [(1, 128, 256), (200, 384, 512), (130, 640, 768), (385, 256, 256)]
+
+
+@pytest.mark.parametrize("m,n,k", RAGGED, ids=[f"{m}x{n}x{k}" for m, n, k in RAGGED])
+def test_ragged_rows_and_half_column_tiles(gpu, m, n, k):
+    """Row counts that are not multiples of 128 (the last row tile is part zeros and only rows
+    below m are stored) and column counts that end in half a 256-column tile; rows of y past m
+    and the guard bytes after y stay untouched."""
+    x, w = operands(m, n, k, seed=m + 3 * n + k)
+    xd, wd = device_bf16(x, m, k), device_bf16(w, n, k)
+    xq, wq = nv.quantize_for_gemm(xd), nv.quantize_for_gemm(wd)
+    ybuf = torch.full((m * n + 1024,), float("nan"), dtype=torch.float32, device="cuda")
+    y = ybuf[: m * n].view(m, n)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_gemm(xq[0], xq[1], xq[2], wq[0], wq[1], wq[2], m, n, k, y, status)
+    y2 = nv.gemm_quantize_x(xd, wq)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.isnan(ybuf[m * n:]).all(), "write past the end of y"
+    assert torch.equal(y.view(torch.int32), y2.view(torch.int32))
+    xc, xs, xt = oracle_quant(x, m, k, "four_over_six", "mse")
+    wc, ws, wt = oracle_quant(w, n, k, "four_over_six", "mse")
+    want = O.gemm_nvfp4(xc, xs, xt, wc, ws, wt, m, n, k)
+    s = O.gemm_nvfp4(magnitude(xc), xs, xt, magnitude(wc), ws, wt, m, n, k)
+    got = y.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - want) <= (k / 64 + 4) * 2.0 ** -22 * s + 1e-30)
