@@ -15,14 +15,16 @@
 //   warp 0 (one lane)  TMA: B codes (and A codes when pre-quantized) as 128-byte swizzled
 //                      tiles, and the operands' 512-byte scale tiles as bulk copies, all
 //                      completing on the stage's "full" mbarrier;
-//   warps 2-7          (prologue variant) quantize the stage's 128 x 256 BF16 activations
+//   warps 6-10         (prologue variant) quantize the stage's 128 x 256 BF16 activations
 //                      into the swizzled A tile and its scale tiles, then arrive on "full";
-//   warp 1 (one lane)  waits for "full", copies the scale tiles into tensor memory
-//                      (tcgen05.cp.32x128b.warpx4), issues four
+//   last warp (lane 0) waits for "full", copies the stage's scale tiles into tensor memory
+//                      (tcgen05.cp.32x128b.warpx4) and commits the copies to the stage's
+//                      "sfready" mbarrier;
+//   warp 1 (one lane)  waits for "sfready", issues four
 //                      tcgen05.mma.kind::mxf4nvf4.block_scale.block16 into the FP32
 //                      accumulator in tensor memory, and commits them to the stage's "empty"
 //                      mbarrier, which releases the slot to the producers.
-// The epilogue (warps 0-3, one 32-lane quarter of tensor memory each) reads the accumulator
+// The epilogue (warps 2-5, one 32-lane quarter of tensor memory each) reads the accumulator
 // with tcgen05.ld and scales it by alpha_x * alpha_w. Every mbarrier wait is bounded: on
 // timeout the kernel records NVFP4_GEMM_TIMEOUT in the status word, every role stops, the
 // CTA frees its tensor memory and returns.
@@ -40,7 +42,7 @@ using namespace nvfp4;
 
 constexpr int kBM = 128, kBN = 256, kBK = 256;    // CTA tile and K slice (elements)
 constexpr int kStages = 4;
-constexpr int kQuantWarps = 6;                    // prologue variant: warps 2..7
+constexpr int kQuantWarps = 5;                    // prologue variant: warps 6..10
 constexpr uint32_t kTmemCols = 512;
 // tensor memory: accumulator columns 0..255; per stage, A scales 4 x 4 columns from 256 and
 // B scales 4 x 8 columns from 320
@@ -248,19 +250,20 @@ struct GemmParams {
 // tile order (tm = t / (n / 256), tn = t % (n / 256)). tmap_a / tmap_b: the codes of x / w as
 // [rows, k/2] byte matrices, boxes of 128 bytes x 128 (A) or 256 (B) rows, 128-byte swizzle
 // (tmap_a unused in the prologue variant). Warps: 0 producer lane, 1 MMA lane (and tensor-memory
-// allocation), 2-5 epilogue (tensor-memory lane quarter = warp % 4), 6-11 quantizers (prologue
-// variant). The ring of K slices runs on across tiles, so the next tile's operands stream in
+// allocation), 2-5 epilogue (tensor-memory lane quarter = warp % 4), 6-10 quantizers (prologue
+// variant), and the last warp's lane 0 copies each slice's scales into tensor memory. The
+// ring of K slices runs on across tiles, so the next tile's operands stream in
 // while the epilogue drains the accumulator; the MMA lane waits for "accumulator empty" (the
 // four epilogue warps) before a tile's first MMA.
 template <bool QUANT>
-constexpr int gemm_threads() { return QUANT ? 384 : 192; }
+__host__ __device__ constexpr int gemm_threads() { return 32 * (6 + (QUANT ? kQuantWarps : 0) + 1); }
 
 template <bool QUANT, bool FOUR, int RULE>
 __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full[kStages], empty[kStages], acc_full, acc_empty, drain;
+    __shared__ __align__(8) uint64_t full[kStages], empty[kStages], sfready[kStages], acc_full, acc_empty, drain;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile uint32_t stop_sh;
     __shared__ float2 tab[128];
@@ -272,14 +275,16 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
     // in a half tile (its second 128 rows of B are zeros and its columns are not stored)
     const int64_t ntn = (p.n + kBN - 1) / kBN, ntiles = ((p.m + kBM - 1) / kBM) * ntn;
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    const uint32_t full0 = smem_u32(&full[0]), empty0 = smem_u32(&empty[0]);
+    const uint32_t full0 = smem_u32(&full[0]), empty0 = smem_u32(&empty[0]), sfr0 = smem_u32(&sfready[0]);
     const uint32_t accf = smem_u32(&acc_full), acce = smem_u32(&acc_empty), drain_bar = smem_u32(&drain);
+    constexpr int kSfWarp = gemm_threads<QUANT>() / 32 - 1;
 
     if (warp == 1) tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(full0 + 8 * s, QUANT ? 1 + kQuantWarps : 1);
             mbar_init(empty0 + 8 * s, 1);
+            mbar_init(sfr0 + 8 * s, 1);
         }
         mbar_init(accf, 1);
         mbar_init(acce, 4);
@@ -333,8 +338,6 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
             const int64_t my_tiles = (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
             const int64_t total = my_tiles * nk;
             const uint64_t dA0 = smem_desc_sw128(sbase), dB0 = smem_desc_sw128(sbase + kABytes);
-            const uint64_t dSA0 = smem_desc(sbase + kABytes + kBBytes, 16, 128);
-            const uint64_t dSB0 = smem_desc(sbase + kABytes + kBBytes + kSfaBytes, 16, 128);
             constexpr uint64_t kSlot = kStageBytes >> 4;   // descriptor start-address units per slot
             int64_t gg = 0;
             int ks = 0, tile_j = 0;
@@ -350,18 +353,12 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
                             break;
                         }
                     }
-                    if (!mbar_wait(full0 + 8 * s, phase)) {
+                    if (!mbar_wait(sfr0 + 8 * s, phase)) {   // operands landed and scales copied
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t ca = tmem + kColSfa + 16 * s, cb = tmem + kColSfb + 32 * s;
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        tmem_copy_sf(ca + 4 * jj, dSA0 + s * kSlot + 32 * jj);
-                        tmem_copy_sf(cb + 8 * jj, dSB0 + s * kSlot + 32 * jj);                 // B rows 0..127
-                        tmem_copy_sf(cb + 8 * jj + 4, dSB0 + s * kSlot + 128 + 32 * jj);       // 128..255
-                    }
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj)
                         mma_fp4(tmem, dA0 + s * kSlot + 2 * jj, dB0 + s * kSlot + 2 * jj, kIdesc, ca + 4 * jj,
@@ -379,6 +376,41 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
             if (!ok) stop_sh = 1;
             mma_commit(drain_bar);   // arrives when every MMA issued above has completed
             if (!mbar_wait(drain_bar, 0)) stop_sh = 1;
+        }
+    } else if (warp == kSfWarp) {
+        if (lane == 0) {   // scale copies into tensor memory, one slice at a time, off the MMA lane
+            const int64_t my_tiles = (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
+            const int64_t total = my_tiles * nk;
+            const uint64_t dSA0 = smem_desc(sbase + kABytes + kBBytes, 16, 128);
+            const uint64_t dSB0 = smem_desc(sbase + kABytes + kBBytes + kSfaBytes, 16, 128);
+            constexpr uint64_t kSlot = kStageBytes >> 4;
+            int64_t gg = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            while (gg < total && ok) {
+#pragma unroll
+                for (int s = 0; s < kStages; ++s) {
+                    if (gg >= total) break;
+                    // slice gg's "full" completes only after the MMAs that last read this slot's
+                    // scale columns have finished (the producer refilled the slot after "empty")
+                    if (!mbar_wait(full0 + 8 * s, phase)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t ca = tmem + kColSfa + 16 * s, cb = tmem + kColSfb + 32 * s;
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        tmem_copy_sf(ca + 4 * jj, dSA0 + s * kSlot + 32 * jj);
+                        tmem_copy_sf(cb + 8 * jj, dSB0 + s * kSlot + 32 * jj);             // B rows 0..127
+                        tmem_copy_sf(cb + 8 * jj + 4, dSB0 + s * kSlot + 128 + 32 * jj);   // 128..255
+                    }
+                    mma_commit(sfr0 + 8 * s);   // "scales ready" once these copies have completed
+                    ++gg;
+                }
+                phase ^= 1;
+            }
+            if (!ok) stop_sh = 1;
         }
     } else if (warp < 6) {   // epilogue: warps 2-5 read tensor-memory lane quarters 2, 3, 0, 1
         const int q = warp & 3;
@@ -428,7 +460,7 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
                 for (int e = 0; e < 64; e += 8) st_v8f(yr + 192 + e, r1 + e, alpha);
             }
         }
-    } else if (QUANT) {   // warps 6-11: quantize each slice's activations into the A tile
+    } else if (QUANT) {   // warps 6-10: quantize each slice's activations into the A tile
         const int qt = tid - 192;
         int g = 0;
         for (int64_t t = blockIdx.x; t < ntiles && !stop_sh; t += gridDim.x) {
