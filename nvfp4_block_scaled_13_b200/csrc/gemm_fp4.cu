@@ -24,8 +24,9 @@
 //                      tcgen05.mma.kind::mxf4nvf4.block_scale.block16 into the FP32
 //                      accumulator in tensor memory, and commits them to the stage's "empty"
 //                      mbarrier, which releases the slot to the producers.
-// The epilogue (warps 2-5, one 32-lane quarter of tensor memory each) reads the accumulator
-// with tcgen05.ld and scales it by alpha_x * alpha_w. Every mbarrier wait is bounded: on
+// The epilogue (warps 2-9, two per 32-lane quarter of tensor memory and 128 columns each; in
+// the prologue variant warps 2-5, one per quarter) reads the accumulator with tcgen05.ld,
+// releases it to the MMA lane and scales it by alpha_x * alpha_w while it stores. Every mbarrier wait is bounded: on
 // timeout the kernel records NVFP4_GEMM_TIMEOUT in the status word, every role stops, the
 // CTA frees its tensor memory and returns.
 #include <cuda.h>
@@ -250,13 +251,18 @@ struct GemmParams {
 // tile order (tm = t / (n / 256), tn = t % (n / 256)). tmap_a / tmap_b: the codes of x / w as
 // [rows, k/2] byte matrices, boxes of 128 bytes x 128 (A) or 256 (B) rows, 128-byte swizzle
 // (tmap_a unused in the prologue variant). Warps: 0 producer lane, 1 MMA lane (and tensor-memory
-// allocation), 2-5 epilogue (tensor-memory lane quarter = warp % 4), 6-10 quantizers (prologue
-// variant), and the last warp's lane 0 copies each slice's scales into tensor memory. The
+// allocation), 2-9 epilogue (2-5 in the prologue variant; tensor-memory lane quarter = warp % 4),
+// 6-10 quantizers (prologue variant), and the last warp's lane 0 copies each slice's scales into
+// tensor memory. The
 // ring of K slices runs on across tiles, so the next tile's operands stream in
-// while the epilogue drains the accumulator; the MMA lane waits for "accumulator empty" (the
-// four epilogue warps) before a tile's first MMA.
+// while the epilogue drains the accumulator; the MMA lane waits for "accumulator empty" (all
+// epilogue warps) before a tile's first MMA.
+// epilogue warps: eight (two per tensor-memory lane quarter, 128 columns each) when operands come
+// in quantized; four in the prologue variant, whose quantizer warps need the registers
 template <bool QUANT>
-__host__ __device__ constexpr int gemm_threads() { return 32 * (6 + (QUANT ? kQuantWarps : 0) + 1); }
+__host__ __device__ constexpr int epi_warps() { return QUANT ? 4 : 8; }
+template <bool QUANT>
+__host__ __device__ constexpr int gemm_threads() { return 32 * (2 + epi_warps<QUANT>() + (QUANT ? kQuantWarps : 0) + 1); }
 
 template <bool QUANT, bool FOUR, int RULE>
 __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
@@ -287,7 +293,7 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
             mbar_init(sfr0 + 8 * s, 1);
         }
         mbar_init(accf, 1);
-        mbar_init(acce, 4);
+        mbar_init(acce, epi_warps<QUANT>());
         mbar_init(drain_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         stop_sh = 0;
@@ -412,7 +418,7 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
             }
             if (!ok) stop_sh = 1;
         }
-    } else if (warp < 6) {   // epilogue: warps 2-5 read tensor-memory lane quarters 2, 3, 0, 1
+    } else if (warp < 2 + epi_warps<QUANT>()) {   // epilogue: warp w reads tensor-memory lane quarter w % 4
         const int q = warp & 3;
         int j = 0;
         for (int64_t t = blockIdx.x; t < ntiles && !stop_sh; t += gridDim.x, ++j) {
@@ -429,35 +435,53 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
             const bool row_ok = row < p.m, full_n = tn * kBN + kBN <= p.n;
             float* yr = p.y + (row_ok ? row : 0) * p.n + tn * kBN;
             const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16);
-            // four chunks of 64 columns: the next chunk's load is in flight while this one is
-            // stored, and the accumulator is released as soon as the last load has landed
             uint32_t r0[64], r1[64];
-            tmem_ld64(trow, r0);
-            tmem_wait_ld();
-            tmem_ld64(trow + 64, r1);
-            if (row_ok) {
+            if constexpr (epi_warps<QUANT>() == 8) {
+                // this warp's 128 columns come out of tensor memory in two loads; the accumulator
+                // is released before any store, so the next tile's MMAs overlap all of them
+                const int c0 = (warp - 2) >> 2 ? 128 : 0;
+                tmem_ld64(trow + c0, r0);
+                tmem_ld64(trow + c0 + 64, r1);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acce);
+                if (row_ok && (c0 == 0 || full_n)) {
 #pragma unroll
-                for (int e = 0; e < 64; e += 8) st_v8f(yr + e, r0 + e, alpha);   // whole 32-byte sectors
-            }
-            tmem_wait_ld();
-            tmem_ld64(trow + 128, r0);
-            if (row_ok) {
+                    for (int e = 0; e < 64; e += 8) st_v8f(yr + c0 + e, r0 + e, alpha);   // whole 32-byte sectors
 #pragma unroll
-                for (int e = 0; e < 64; e += 8) st_v8f(yr + 64 + e, r1 + e, alpha);
-            }
-            tmem_wait_ld();
-            tmem_ld64(trow + 192, r1);
-            if (row_ok && full_n) {
+                    for (int e = 0; e < 64; e += 8) st_v8f(yr + c0 + 64 + e, r1 + e, alpha);
+                }
+            } else {
+                // four chunks of 64 columns: the next chunk's load is in flight while this one is
+                // stored, and the accumulator is released as soon as the last load has landed
+                tmem_ld64(trow, r0);
+                tmem_wait_ld();
+                tmem_ld64(trow + 64, r1);
+                if (row_ok) {
 #pragma unroll
-                for (int e = 0; e < 64; e += 8) st_v8f(yr + 128 + e, r0 + e, alpha);
-            }
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acce);
-            if (row_ok && full_n) {
+                    for (int e = 0; e < 64; e += 8) st_v8f(yr + e, r0 + e, alpha);
+                }
+                tmem_wait_ld();
+                tmem_ld64(trow + 128, r0);
+                if (row_ok) {
 #pragma unroll
-                for (int e = 0; e < 64; e += 8) st_v8f(yr + 192 + e, r1 + e, alpha);
+                    for (int e = 0; e < 64; e += 8) st_v8f(yr + 64 + e, r1 + e, alpha);
+                }
+                tmem_wait_ld();
+                tmem_ld64(trow + 192, r1);
+                if (row_ok && full_n) {
+#pragma unroll
+                    for (int e = 0; e < 64; e += 8) st_v8f(yr + 128 + e, r0 + e, alpha);
+                }
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acce);
+                if (row_ok && full_n) {
+#pragma unroll
+                    for (int e = 0; e < 64; e += 8) st_v8f(yr + 192 + e, r1 + e, alpha);
+                }
             }
         }
     } else if (QUANT) {   // warps 6-10: quantize each slice's activations into the A tile
