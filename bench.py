@@ -306,8 +306,9 @@ def run_reference(args, rank, world):
 
 def gemm_leg(nv, torch, dev, peak_tflops, m=8192, n=4096, k=4096, reps=20):
     """The block-scaled FP4 GEMM on a transformer-layer shape (m tokens x k -> n): activations
-    quantized once (Four Over Six, MSE) then nvfp4_gemm, and the variant that quantizes them in
-    its prologue. TFLOP/s = 2 m n k / t against the FP4 dense peak."""
+    quantized once (Four Over Six, MSE) then nvfp4_gemm, the BF16-output variant whose epilogue
+    also finds the result's amax (nvfp4_gemm_bf16), and the variant that quantizes the
+    activations in its prologue. TFLOP/s = 2 m n k / t against the FP4 dense peak."""
     gen = torch.Generator(device=dev).manual_seed(7)
     x = (torch.randn(m, k, device=dev, generator=gen) * torch.exp(torch.randn(k, device=dev, generator=gen))
          ).to(torch.bfloat16)
@@ -316,11 +317,15 @@ def gemm_leg(nv, torch, dev, peak_tflops, m=8192, n=4096, k=4096, reps=20):
     ax = nv.amax(x, 1)
     xq = nv.quantize_for_gemm(x, amax_values=ax)
     y = torch.empty(m, n, dtype=torch.float32, device=dev)
+    y16 = torch.empty(m, n, dtype=torch.bfloat16, device=dev)
+    y_amax = torch.empty(1, dtype=torch.float32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     s = torch.cuda.current_stream(dev).cuda_stream
     legs = {
         "quantize_x": lambda: nv.nvfp4_quantize_gemm(x, m, k, ax, 1, 2, xq[0], xq[1], xq[2], None, s),
         "gemm": lambda: nv.nvfp4_gemm(xq[0], xq[1], xq[2], wq[0], wq[1], wq[2], m, n, k, y, status, s),
+        "gemm_bf16_amax": lambda: nv.nvfp4_gemm_bf16(xq[0], xq[1], xq[2], wq[0], wq[1], wq[2], m, n, k, y16, y_amax,
+                                                     status, s),
         "prologue": lambda: nv.nvfp4_gemm_quantize_x(x, ax, 1, 2, wq[0], wq[1], wq[2], m, n, k, y, status, s),
     }
     ms = {}
@@ -341,8 +346,9 @@ def gemm_leg(nv, torch, dev, peak_tflops, m=8192, n=4096, k=4096, reps=20):
            "peak_tflops": peak_tflops, "frac": round(tf / peak_tflops, 4),
            "quantize_then_gemm_tflops": round(flops / ((ms["gemm"] + ms["quantize_x"]) * 1e-3) / 1e12, 1),
            "prologue_tflops": round(flops / (ms["prologue"] * 1e-3) / 1e12, 1),
+           "bf16_amax_tflops": round(flops / (ms["gemm_bf16_amax"] * 1e-3) / 1e12, 1),
            "status": int(status.item())}
-    del x, w, wq, xq, y
+    del x, w, wq, xq, y, y16
     return out
 
 

@@ -165,23 +165,6 @@ NVFP4_API nvfp4_status nvfp4_quantize_gemm(const uint16_t* x, int64_t rows, int6
                                            nvfp4_mode mode, nvfp4_rule rule, uint8_t* codes, uint8_t* scales,
                                            float* tscale, uint8_t* choice, cudaStream_t stream);
 
-/* Distillation loss of quantization-aware distillation ("Quantization-Aware Distillation for
- * NVFP4 Inference Accuracy Recovery", technical summary §2: the NVFP4 student, whose forward
- * runs through simulated quantization (nvfp4_fakequant), is trained against the frozen BF16
- * teacher with L = D_KL(p_teacher || p_student)). For every row r of [rows, vocab] logits:
- *   p = softmax(teacher[r] / tau), q = softmax(student[r] / tau)
- *   kl[r]      = sum_v p_v (ln p_v - ln q_v)                    (nats)
- *   grad[r, v] = BF16(grad_scale * (q_v - p_v))   (d kl[r] / d student[r, v] = (q_v - p_v) / tau:
- *                pass grad_scale = 1 / (tau * rows) for the gradient of the mean loss)
- *   teacher, student  [rows, vocab] BF16 bits, 2-byte aligned (16-byte aligned rows with
- *                     vocab % 8 == 0 take the vectorised path)                     (in)
- *   kl                [rows] float, 4-byte aligned                                (out)
- *   grad              NULL, or [rows, vocab] BF16 bits, 2-byte aligned            (out)
- * Arithmetic in binary32 with an online (single read) softmax per row and the hardware base-2
- * exponential; the results agree with the binary64 definition to about 1e-6 of the loss's
- * magnitude (tests/test_gpu_5_qad_kl.py states the bounds). tau must be finite and > 0,
- * grad_scale finite (else NVFP4_ERR_VALUE); vocab >= 1; logits must be finite. rows == 0 does
- * nothing. One kernel; a second read of each row when grad is requested. */
 /* Bit set in a GEMM's status word when one of the kernel's bounded waits for the tensor core
  * timed out (about two seconds); the kernel then stops, frees its tensor memory and leaves y
  * partly written. */
@@ -205,6 +188,22 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* x_codes, const uint8_t* x_scale
                                   int64_t m, int64_t n, int64_t k, float* y, uint32_t* status,
                                   cudaStream_t stream);
 
+/* The same GEMM with a BF16 result and, fused into its epilogue, the absolute maximum of that
+ * result: the tensor amax from which the next quantization of y derives its FP32 tensor scale
+ * ("Four Over Six", Implementation details), so that quantizing y takes one pass over it and
+ * no nvfp4_amax read (the reproducible workflow lets the user choose dynamic or static scales:
+ * "NVIDIA、「Nemotron 3.5 Lightning」のNVFP4量子化手法を公開", section on the released workflow).
+ *   y       [m, n] BF16 bits, y[i, j] = BF16 round-to-nearest-even of the binary32 value
+ *           nvfp4_gemm writes at [i, j]; 32-byte aligned                          (out, device)
+ *   y_amax  NULL, or [1] float: max |y| over the BF16 values written, exactly (equal to
+ *           nvfp4_amax of y; NaN if a y is NaN); 4-byte aligned; zero-filled first in stream
+ *           order (cudaMemsetAsync), so an empty product leaves 0                 (out, device)
+ * Operands, shapes, status and errors as nvfp4_gemm. */
+NVFP4_API nvfp4_status nvfp4_gemm_bf16(const uint8_t* x_codes, const uint8_t* x_scales, const float* x_tscale,
+                                       const uint8_t* w_codes, const uint8_t* w_scales, const float* w_tscale,
+                                       int64_t m, int64_t n, int64_t k, uint16_t* y, float* y_amax,
+                                       uint32_t* status, cudaStream_t stream);
+
 /* The same GEMM with the activation operand quantized inside the kernel's prologue from BF16
  * x [m, k] (32-byte aligned) with its amax x_amax [1] (device), in `mode` under `rule`,
  * exactly as nvfp4_quantize_gemm would quantize it (the pages apply Four Over Six to the
@@ -215,6 +214,23 @@ NVFP4_API nvfp4_status nvfp4_gemm_quantize_x(const uint16_t* x, const float* x_a
                                              const float* w_tscale, int64_t m, int64_t n, int64_t k, float* y,
                                              uint32_t* status, cudaStream_t stream);
 
+/* Distillation loss of quantization-aware distillation ("Quantization-Aware Distillation for
+ * NVFP4 Inference Accuracy Recovery", technical summary §2: the NVFP4 student, whose forward
+ * runs through simulated quantization (nvfp4_fakequant), is trained against the frozen BF16
+ * teacher with L = D_KL(p_teacher || p_student)). For every row r of [rows, vocab] logits:
+ *   p = softmax(teacher[r] / tau), q = softmax(student[r] / tau)
+ *   kl[r]      = sum_v p_v (ln p_v - ln q_v)                    (nats)
+ *   grad[r, v] = BF16(grad_scale * (q_v - p_v))   (d kl[r] / d student[r, v] = (q_v - p_v) / tau:
+ *                pass grad_scale = 1 / (tau * rows) for the gradient of the mean loss)
+ *   teacher, student  [rows, vocab] BF16 bits, 2-byte aligned (16-byte aligned rows with
+ *                     vocab % 8 == 0 take the vectorised path)                     (in)
+ *   kl                [rows] float, 4-byte aligned                                (out)
+ *   grad              NULL, or [rows, vocab] BF16 bits, 2-byte aligned            (out)
+ * Arithmetic in binary32 with an online (single read) softmax per row and the hardware base-2
+ * exponential; the results agree with the binary64 definition to about 1e-6 of the loss's
+ * magnitude (tests/test_gpu_5_qad_kl.py states the bounds). tau must be finite and > 0,
+ * grad_scale finite (else NVFP4_ERR_VALUE); vocab >= 1; logits must be finite. rows == 0 does
+ * nothing. One kernel; a second read of each row when grad is requested. */
 NVFP4_API nvfp4_status nvfp4_qad_kl(const uint16_t* teacher, const uint16_t* student, int64_t rows, int64_t vocab,
                                     float tau, float grad_scale, float* kl, uint16_t* grad, cudaStream_t stream);
 

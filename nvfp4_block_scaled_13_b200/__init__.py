@@ -23,9 +23,9 @@ __all__ = [
     "load", "library_path", "Nvfp4Error",
     "SCALE6", "FOUR_OVER_SIX", "RULE_MAXERR", "RULE_MAE", "RULE_MSE",
     "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_quantize_gemm", "nvfp4_qad_kl",
-    "nvfp4_gemm", "nvfp4_gemm_quantize_x", "GEMM_TIMEOUT", "nvfp4_status_string", "nvfp4_version",
+    "nvfp4_gemm", "nvfp4_gemm_bf16", "nvfp4_gemm_quantize_x", "GEMM_TIMEOUT", "nvfp4_status_string", "nvfp4_version",
     "Quantized", "amax", "quantize", "fakequant", "dequantize", "quantize_for_gemm", "gemm_scale_bytes",
-    "qad_kl", "fakequant_ste", "gemm", "gemm_quantize_x",
+    "qad_kl", "fakequant_ste", "gemm", "gemm_bf16", "gemm_quantize_x",
 ]
 
 GEMM_TIMEOUT = 1   # bit of a GEMM's status word: a bounded wait for the tensor core timed out
@@ -66,9 +66,10 @@ def load():
         L.nvfp4_quantize_gemm.argtypes = [vp, i64, i64, vp, i32, i32, vp, vp, vp, vp, vp]
         L.nvfp4_qad_kl.argtypes = [vp, vp, i64, i64, ctypes.c_float, ctypes.c_float, vp, vp, vp]
         L.nvfp4_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp]
+        L.nvfp4_gemm_bf16.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp]
         L.nvfp4_gemm_quantize_x.argtypes = [vp, vp, i32, i32, vp, vp, vp, i64, i64, i64, vp, vp, vp]
         for f in (L.nvfp4_amax, L.nvfp4_quantize, L.nvfp4_dequantize, L.nvfp4_fakequant, L.nvfp4_quantize_gemm,
-                  L.nvfp4_qad_kl, L.nvfp4_gemm, L.nvfp4_gemm_quantize_x):
+                  L.nvfp4_qad_kl, L.nvfp4_gemm, L.nvfp4_gemm_bf16, L.nvfp4_gemm_quantize_x):
             f.restype = i32
         L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
         L.nvfp4_version.argtypes, L.nvfp4_version.restype = [], i32
@@ -139,6 +140,13 @@ def nvfp4_fakequant(x, groups, rows, cols, amax, mode, rule, y, choice=None, str
 def nvfp4_gemm(x_codes, x_scales, x_tscale, w_codes, w_scales, w_tscale, m, n, k, y, status=None, stream=None):
     _check(load().nvfp4_gemm(_ptr(x_codes), _ptr(x_scales), _ptr(x_tscale), _ptr(w_codes), _ptr(w_scales),
                              _ptr(w_tscale), m, n, k, _ptr(y), _ptr(status), _stream(stream)), "nvfp4_gemm")
+
+
+def nvfp4_gemm_bf16(x_codes, x_scales, x_tscale, w_codes, w_scales, w_tscale, m, n, k, y, y_amax=None,
+                    status=None, stream=None):
+    _check(load().nvfp4_gemm_bf16(_ptr(x_codes), _ptr(x_scales), _ptr(x_tscale), _ptr(w_codes), _ptr(w_scales),
+                                  _ptr(w_tscale), m, n, k, _ptr(y), _ptr(y_amax), _ptr(status), _stream(stream)),
+           "nvfp4_gemm_bf16")
 
 
 def nvfp4_gemm_quantize_x(x, x_amax, mode, rule, w_codes, w_scales, w_tscale, m, n, k, y, status=None,
@@ -276,6 +284,22 @@ def gemm(xq, wq, stream=None):
     if int(status.item()) & GEMM_TIMEOUT:
         raise Nvfp4Error("nvfp4_gemm: a wait for the tensor core timed out")
     return y
+
+
+def gemm_bf16(xq, wq, stream=None):
+    """(y, y_amax): y = Xq Wq^T rounded to BF16 and its absolute maximum [1] (float32), found in
+    the GEMM's epilogue, ready to be the amax of y's own quantization."""
+    import torch
+
+    (xc, xs, xt, _), (wc, ws, wt, _) = xq, wq
+    m, n, k = xc.shape[0], wc.shape[0], 2 * xc.shape[1]
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=xc.device)
+    y_amax = torch.empty(1, dtype=torch.float32, device=xc.device)
+    status = torch.zeros(1, dtype=torch.int32, device=xc.device)
+    nvfp4_gemm_bf16(xc, xs, xt, wc, ws, wt, m, n, k, y, y_amax, status, stream)
+    if int(status.item()) & GEMM_TIMEOUT:
+        raise Nvfp4Error("nvfp4_gemm_bf16: a wait for the tensor core timed out")
+    return y, y_amax
 
 
 def gemm_quantize_x(x, wq, mode="four_over_six", rule="mse", amax_values=None, stream=None):

@@ -221,6 +221,23 @@ __device__ __forceinline__ void st_v8f(float* dst, const uint32_t* r, float alph
                  : "memory");
 }
 
+// 16 consecutive outputs as BF16 (one 32-byte sector), each accumulator word times alpha rounded
+// to binary32 and then to BF16 (so each equals the BF16 rounding of the FP32 output). `mag`
+// collects the largest |alpha * acc| as binary32 bits: non-negative floats order like their
+// bits, and a NaN sorts above infinity.
+__device__ __forceinline__ void st_v16bf(uint16_t* dst, const uint32_t* r, float alpha, uint32_t& mag) {
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float a = __uint_as_float(r[2 * i]) * alpha, b = __uint_as_float(r[2 * i + 1]) * alpha;
+        mag = max(mag, max(__float_as_uint(a) & 0x7FFFFFFFu, __float_as_uint(b) & 0x7FFFFFFFu));
+        w[i] = bf16x2(make_float2(a, b));
+    }
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                 "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
+
 __device__ __forceinline__ void sts16(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
@@ -242,7 +259,9 @@ struct GemmParams {
     const float* x_tscale;    // pre-quantized variant: alpha_x, [1]
     const uint8_t* w_scales;  // tiled scales of w
     const float* w_tscale;    // alpha_w, [1]
-    float* y;                 // [m, n]
+    float* y;                 // [m, n] FP32, or
+    uint16_t* y16;            // [m, n] BF16 (nvfp4_gemm_bf16)
+    float* y_amax;            // nullable, nvfp4_gemm_bf16: max |y|, zero-filled before the launch
     uint32_t* status;         // nullable; NVFP4_GEMM_TIMEOUT is or-ed in on a timed-out wait
     int64_t m, n, k;
 };
@@ -264,10 +283,11 @@ __host__ __device__ constexpr int epi_warps() { return QUANT ? 4 : 8; }
 template <bool QUANT>
 __host__ __device__ constexpr int gemm_threads() { return 32 * (2 + epi_warps<QUANT>() + (QUANT ? kQuantWarps : 0) + 1); }
 
-template <bool QUANT, bool FOUR, int RULE>
+template <bool QUANT, bool FOUR, int RULE, bool BF16 = false>
 __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const GemmParams p) {
+    static_assert(!(QUANT && BF16), "the BF16 output is built for pre-quantized operands");
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full[kStages], empty[kStages], sfready[kStages], acc_full, acc_empty, drain;
     __shared__ uint32_t tmem_base_sh;
@@ -433,7 +453,7 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
             const float alpha = (QUANT ? gc.alpha : __ldg(p.x_tscale)) * __ldg(p.w_tscale);
             const int64_t row = tm * kBM + 32 * q + lane;
             const bool row_ok = row < p.m, full_n = tn * kBN + kBN <= p.n;
-            float* yr = p.y + (row_ok ? row : 0) * p.n + tn * kBN;
+            float* yr = BF16 ? nullptr : p.y + (row_ok ? row : 0) * p.n + tn * kBN;
             const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16);
             uint32_t r0[64], r1[64];
             if constexpr (epi_warps<QUANT>() == 8) {
@@ -446,7 +466,25 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(acce);
-                if (row_ok && (c0 == 0 || full_n)) {
+                if constexpr (BF16) {
+                    // BF16 output with its amax fused in: rounding is monotone and symmetric, so
+                    // max |BF16(v)| = BF16(max |v|), one rounding per warp and tile
+                    uint32_t mag = 0;
+                    if (row_ok && (c0 == 0 || full_n)) {
+                        uint16_t* yb = p.y16 + (row_ok ? row : 0) * p.n + tn * kBN + c0;
+#pragma unroll
+                        for (int e = 0; e < 64; e += 16) st_v16bf(yb + e, r0 + e, alpha, mag);
+#pragma unroll
+                        for (int e = 0; e < 64; e += 16) st_v16bf(yb + 64 + e, r1 + e, alpha, mag);
+                    }
+                    if (p.y_amax != nullptr) {
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) mag = max(mag, __shfl_xor_sync(0xFFFFFFFFu, mag, o));
+                        if (lane == 0 && mag != 0)
+                            atomicMax(reinterpret_cast<unsigned int*>(p.y_amax),
+                                      __float_as_uint(__bfloat162float(__float2bfloat16_rn(__uint_as_float(mag)))));
+                    }
+                } else if (row_ok && (c0 == 0 || full_n)) {
 #pragma unroll
                     for (int e = 0; e < 64; e += 8) st_v8f(yr + c0 + e, r0 + e, alpha);   // whole 32-byte sectors
 #pragma unroll
@@ -570,9 +608,9 @@ bool codes_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_byt
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool QUANT, bool FOUR, int RULE>
+template <bool QUANT, bool FOUR, int RULE, bool BF16 = false>
 nvfp4_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& p, cudaStream_t stream) {
-    auto kernel = gemm_fp4_kernel<QUANT, FOUR, RULE>;
+    auto kernel = gemm_fp4_kernel<QUANT, FOUR, RULE, BF16>;
     // per device, so set on every launch (cheap)
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem) != cudaSuccess)
         return NVFP4_ERR_CUDA;
@@ -597,18 +635,29 @@ nvfp4_status check_gemm_shape(int64_t m, int64_t n, int64_t k) {
 
 }  // namespace
 
-extern "C" nvfp4_status nvfp4_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const float* x_tscale,
-                                   const uint8_t* w_codes, const uint8_t* w_scales, const float* w_tscale,
-                                   int64_t m, int64_t n, int64_t k, float* y, uint32_t* status,
-                                   cudaStream_t stream) {
+namespace {
+
+// nvfp4_gemm and nvfp4_gemm_bf16: exactly one of y (FP32) and y16 (BF16) is set.
+nvfp4_status gemm_prequantized(const uint8_t* x_codes, const uint8_t* x_scales, const float* x_tscale,
+                               const uint8_t* w_codes, const uint8_t* w_scales, const float* w_tscale, int64_t m,
+                               int64_t n, int64_t k, float* y, uint16_t* y16, float* y_amax, uint32_t* status,
+                               cudaStream_t stream) {
     const nvfp4_status st = check_gemm_shape(m, n, k);
     if (st != NVFP4_OK) return st;
-    if (m == 0 || n == 0) return NVFP4_OK;
-    if (!x_codes || !x_scales || !x_tscale || !w_codes || !w_scales || !w_tscale || !y) return NVFP4_ERR_NULL;
-    if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
-        (reinterpret_cast<uintptr_t>(y) & 31u) || !aligned4(x_tscale) || !aligned4(w_tscale) || !aligned4(status))
-        return NVFP4_ERR_ALIGN;
-    if (k == 0) return NVFP4_ERR_SHAPE;
+    if (y_amax != nullptr && !aligned4(y_amax)) return NVFP4_ERR_ALIGN;
+    const bool empty = m == 0 || n == 0;
+    if (!empty) {
+        if (!x_codes || !x_scales || !x_tscale || !w_codes || !w_scales || !w_tscale || (!y && !y16))
+            return NVFP4_ERR_NULL;
+        const uintptr_t yp = y != nullptr ? reinterpret_cast<uintptr_t>(y) : reinterpret_cast<uintptr_t>(y16);
+        if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+            (yp & 31u) || !aligned4(x_tscale) || !aligned4(w_tscale) || !aligned4(status))
+            return NVFP4_ERR_ALIGN;
+        if (k == 0) return NVFP4_ERR_SHAPE;
+    }
+    // the amax is an atomic maximum over the tiles: it starts from +0 in stream order
+    if (y_amax != nullptr && cudaMemsetAsync(y_amax, 0, sizeof(float), stream) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (empty) return NVFP4_OK;
     CUtensorMap ma, mb;
     if (!codes_map(&ma, x_codes, m, k / 2, kBM) || !codes_map(&mb, w_codes, n, k / 2, kBN)) return NVFP4_ERR_CUDA;
     GemmParams p{};
@@ -617,11 +666,32 @@ extern "C" nvfp4_status nvfp4_gemm(const uint8_t* x_codes, const uint8_t* x_scal
     p.w_scales = w_scales;
     p.w_tscale = w_tscale;
     p.y = y;
+    p.y16 = y16;
+    p.y_amax = y_amax;
     p.status = status;
     p.m = m;
     p.n = n;
     p.k = k;
+    if (y16 != nullptr) return launch_gemm<false, true, kMse, true>(ma, mb, p, stream);
     return launch_gemm<false, true, kMse>(ma, mb, p, stream);
+}
+
+}  // namespace
+
+extern "C" nvfp4_status nvfp4_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const float* x_tscale,
+                                   const uint8_t* w_codes, const uint8_t* w_scales, const float* w_tscale,
+                                   int64_t m, int64_t n, int64_t k, float* y, uint32_t* status,
+                                   cudaStream_t stream) {
+    return gemm_prequantized(x_codes, x_scales, x_tscale, w_codes, w_scales, w_tscale, m, n, k, y, nullptr, nullptr,
+                             status, stream);
+}
+
+extern "C" nvfp4_status nvfp4_gemm_bf16(const uint8_t* x_codes, const uint8_t* x_scales, const float* x_tscale,
+                                        const uint8_t* w_codes, const uint8_t* w_scales, const float* w_tscale,
+                                        int64_t m, int64_t n, int64_t k, uint16_t* y, float* y_amax,
+                                        uint32_t* status, cudaStream_t stream) {
+    return gemm_prequantized(x_codes, x_scales, x_tscale, w_codes, w_scales, w_tscale, m, n, k, nullptr, y, y_amax,
+                             status, stream);
 }
 
 extern "C" nvfp4_status nvfp4_gemm_quantize_x(const uint16_t* x, const float* x_amax, nvfp4_mode mode,

@@ -7,6 +7,7 @@ Student-t(3)-like tails times a lognormal per-channel scale, weights w [n, k] BF
 The weights are quantized once (Four Over Six, MSE). Reported, as mean CUDA-event times over
 `reps` launches after warm-up, with TFLOP/s = 2 m n k / t:
   gemm         nvfp4_gemm on pre-quantized activations,
+  gemm_bf16    nvfp4_gemm_bf16 (BF16 result and its amax from the epilogue),
   quantize_x   nvfp4_quantize_gemm of the activations (amax given),
   prologue     nvfp4_gemm_quantize_x (activations quantized inside the GEMM).
 """
@@ -42,11 +43,16 @@ def main():
     ax = nv.amax(x, 1)
     xq = nv.quantize_for_gemm(x, a.mode, a.rule, amax_values=ax)
     y = torch.empty(a.m, a.n, dtype=torch.float32, device="cuda")
+    y16 = torch.empty(a.m, a.n, dtype=torch.bfloat16, device="cuda")
+    y_amax = torch.empty(1, dtype=torch.float32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     s = torch.cuda.current_stream().cuda_stream
 
     def run_gemm():
         nv.nvfp4_gemm(xq[0], xq[1], xq[2], wq[0], wq[1], wq[2], a.m, a.n, a.k, y, status, s)
+
+    def run_gemm_bf16():
+        nv.nvfp4_gemm_bf16(xq[0], xq[1], xq[2], wq[0], wq[1], wq[2], a.m, a.n, a.k, y16, y_amax, status, s)
 
     def run_quant():
         nv.nvfp4_quantize_gemm(x, a.m, a.k, ax, a.mode, a.rule, xq[0], xq[1], xq[2], None, s)
@@ -56,7 +62,8 @@ def main():
 
     flops = 2.0 * a.m * a.n * a.k
     out = {"m": a.m, "n": a.n, "k": a.k, "mode": a.mode, "rule": a.rule}
-    for name, fn in (("gemm", run_gemm), ("quantize_x", run_quant), ("prologue", run_prologue)):
+    for name, fn in (("gemm", run_gemm), ("gemm_bf16", run_gemm_bf16), ("quantize_x", run_quant),
+                     ("prologue", run_prologue)):
         for _ in range(3):
             fn()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

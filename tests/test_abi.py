@@ -19,7 +19,7 @@ def header_functions(path):
 
 def test_header_declares_the_boundary():
     names = header_functions(os.path.join(ROOT, "include", "nvfp4.h"))
-    assert names == ["nvfp4_amax", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_gemm", "nvfp4_gemm_quantize_x",
+    assert names == ["nvfp4_amax", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_gemm", "nvfp4_gemm_bf16", "nvfp4_gemm_quantize_x",
                      "nvfp4_qad_kl", "nvfp4_quantize", "nvfp4_quantize_gemm", "nvfp4_status_string",
                      "nvfp4_version"]
 
@@ -98,6 +98,14 @@ A = 1 << 20          # 32-byte aligned
     (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 128, 256, 256, A, A + 2, None), 3),
     (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 128, 256, 256, A + 16, None, None), 3),
     (lambda L: L.nvfp4_gemm(A, A, A, A, A, A, 0, 256, 256, None, None, None), 0),
+    # nvfp4_gemm_bf16(xc, xs, xt, wc, ws, wt, m, n, k, y, y_amax, status, stream)
+    (lambda L: L.nvfp4_gemm_bf16(A, A, A, A, A, A, 128, 256, 200, A, A, None, None), 2),
+    (lambda L: L.nvfp4_gemm_bf16(A, A, A, A, A, A, 128, 192, 256, A, A, None, None), 2),
+    (lambda L: L.nvfp4_gemm_bf16(None, A, A, A, A, A, 128, 256, 256, A, A, None, None), 1),
+    (lambda L: L.nvfp4_gemm_bf16(A, A, A, A, A, A, 128, 256, 256, None, A, None, None), 1),
+    (lambda L: L.nvfp4_gemm_bf16(A, A, A, A, A, A, 128, 256, 256, A + 16, A, None, None), 3),
+    (lambda L: L.nvfp4_gemm_bf16(A, A, A, A, A, A, 128, 256, 256, A, A + 2, None, None), 3),
+    (lambda L: L.nvfp4_gemm_bf16(A, A, A, A, A, A, 0, 256, 256, None, None, None, None), 0),
     # nvfp4_gemm_quantize_x(x, amax, mode, rule, wc, ws, wt, m, n, k, y, status, stream)
     (lambda L: L.nvfp4_gemm_quantize_x(A, A, 2, 2, A, A, A, 128, 256, 256, A, None, None), 4),
     (lambda L: L.nvfp4_gemm_quantize_x(A, A, 1, 3, A, A, A, 128, 256, 256, A, None, None), 5),
