@@ -17,9 +17,10 @@
 //                      completing on the stage's "full" mbarrier;
 //   warps 6-10         (prologue variant) quantize the stage's 128 x 256 BF16 activations
 //                      into the swizzled A tile and its scale tiles, then arrive on "full";
-//   last warp (lane 0) waits for "full", copies the stage's scale tiles into tensor memory
-//                      (tcgen05.cp.32x128b.warpx4) and commits the copies to the stage's
-//                      "sfready" mbarrier;
+//   last warps (lane 0; two, or one in the prologue variant) wait for "full", copy the
+//                      stage's scale tiles into tensor memory (tcgen05.cp.32x128b.warpx4, each
+//                      lane those of its share of the four MMAs) and commit the copies to the
+//                      stage's "sfready" mbarrier;
 //   warp 1 (one lane)  waits for "sfready", issues four
 //                      tcgen05.mma.kind::mxf4nvf4.block_scale.block16 into the FP32
 //                      accumulator in tensor memory, and commits them to the stage's "empty"
@@ -271,8 +272,8 @@ struct GemmParams {
 // [rows, k/2] byte matrices, boxes of 128 bytes x 128 (A) or 256 (B) rows, 128-byte swizzle
 // (tmap_a unused in the prologue variant). Warps: 0 producer lane, 1 MMA lane (and tensor-memory
 // allocation), 2-9 epilogue (2-5 in the prologue variant; tensor-memory lane quarter = warp % 4),
-// 6-10 quantizers (prologue variant), and the last warp's lane 0 copies each slice's scales into
-// tensor memory. The
+// 6-10 quantizers (prologue variant), and lane 0 of the last warps (10-11; 11 in the prologue
+// variant) copies each slice's scales into tensor memory. The
 // ring of K slices runs on across tiles, so the next tile's operands stream in
 // while the epilogue drains the accumulator; the MMA lane waits for "accumulator empty" (all
 // epilogue warps) before a tile's first MMA.
@@ -280,8 +281,14 @@ struct GemmParams {
 // in quantized; four in the prologue variant, whose quantizer warps need the registers
 template <bool QUANT>
 __host__ __device__ constexpr int epi_warps() { return QUANT ? 4 : 8; }
+// scale-copy warps (the last ones): two when operands come in quantized, each issuing the
+// copies of two of a slice's four MMAs; one in the prologue variant
 template <bool QUANT>
-__host__ __device__ constexpr int gemm_threads() { return 32 * (2 + epi_warps<QUANT>() + (QUANT ? kQuantWarps : 0) + 1); }
+__host__ __device__ constexpr int sf_warps() { return QUANT ? 1 : 2; }
+template <bool QUANT>
+__host__ __device__ constexpr int gemm_threads() {
+    return 32 * (2 + epi_warps<QUANT>() + (QUANT ? kQuantWarps : 0) + sf_warps<QUANT>());
+}
 
 template <bool QUANT, bool FOUR, int RULE, bool BF16 = false>
 __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
@@ -303,14 +310,14 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t full0 = smem_u32(&full[0]), empty0 = smem_u32(&empty[0]), sfr0 = smem_u32(&sfready[0]);
     const uint32_t accf = smem_u32(&acc_full), acce = smem_u32(&acc_empty), drain_bar = smem_u32(&drain);
-    constexpr int kSfWarp = gemm_threads<QUANT>() / 32 - 1;
+    constexpr int kSfWarp0 = gemm_threads<QUANT>() / 32 - sf_warps<QUANT>();   // first scale-copy warp
 
     if (warp == 1) tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(full0 + 8 * s, QUANT ? 1 + kQuantWarps : 1);
             mbar_init(empty0 + 8 * s, 1);
-            mbar_init(sfr0 + 8 * s, 1);
+            mbar_init(sfr0 + 8 * s, sf_warps<QUANT>());
         }
         mbar_init(accf, 1);
         mbar_init(acce, epi_warps<QUANT>());
@@ -403,8 +410,10 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
             mma_commit(drain_bar);   // arrives when every MMA issued above has completed
             if (!mbar_wait(drain_bar, 0)) stop_sh = 1;
         }
-    } else if (warp == kSfWarp) {
+    } else if (warp >= kSfWarp0) {
         if (lane == 0) {   // scale copies into tensor memory, one slice at a time, off the MMA lane
+            constexpr int kPer = 4 / sf_warps<QUANT>();   // MMAs whose scales this lane copies
+            const int j0 = (warp - kSfWarp0) * kPer;
             const int64_t my_tiles = (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
             const int64_t total = my_tiles * nk;
             const uint64_t dSA0 = smem_desc(sbase + kABytes + kBBytes, 16, 128);
@@ -426,7 +435,8 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
                     tc_fence_after();
                     const uint32_t ca = tmem + kColSfa + 16 * s, cb = tmem + kColSfb + 32 * s;
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
+                    for (int i = 0; i < kPer; ++i) {
+                        const int jj = j0 + i;
                         tmem_copy_sf(ca + 4 * jj, dSA0 + s * kSlot + 32 * jj);
                         tmem_copy_sf(cb + 8 * jj, dSB0 + s * kSlot + 32 * jj);             // B rows 0..127
                         tmem_copy_sf(cb + 8 * jj + 4, dSB0 + s * kSlot + 128 + 32 * jj);   // 128..255
