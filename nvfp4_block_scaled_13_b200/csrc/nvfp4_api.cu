@@ -39,9 +39,11 @@ int sm_count() {
     return n;
 }
 
-// Resident CTAs per SM for a kernel, cached per kernel instantiation and device.
-template <typename Kernel>
-int ctas_per_sm(Kernel kernel) {
+// Resident CTAs per SM for a kernel, cached per kernel and device. The kernel is a template
+// argument so that every kernel gets its own cache: the quantizer's instantiations share one
+// function type, and a cache keyed by the type would hand one kernel's occupancy to another.
+template <auto kernel>
+int ctas_per_sm() {
     static std::atomic<int> cache[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
@@ -54,9 +56,9 @@ int ctas_per_sm(Kernel kernel) {
 }
 
 // Persistent grid: enough CTAs to fill every SM at full occupancy, never more than the work.
-template <typename Kernel>
-unsigned grid_for(Kernel kernel, int64_t work_items) {
-    const int64_t full = static_cast<int64_t>(sm_count()) * ctas_per_sm(kernel);
+template <auto kernel>
+unsigned grid_for(int64_t work_items) {
+    const int64_t full = static_cast<int64_t>(sm_count()) * ctas_per_sm<kernel>();
     const int64_t need = (work_items + kThreads - 1) / kThreads;
     const int64_t g = need < full ? need : full;
     return static_cast<unsigned>(g < 1 ? 1 : g);
@@ -130,12 +132,12 @@ nvfp4_status launch_quant(const nvfp4::QuantParams& p, cudaStream_t stream) {
     const bool grouped = (p.groups == 1 || bpg % 32 == 0) && bpg < (int64_t(1) << 30);
     if (grouped) {
         // CTAs work inside one group at a time, with the group's scale table in shared memory
-        auto kernel = nvfp4::quantize_grouped_kernel<FOUR, RULE, FQ>;
-        const dim3 grid = grouped_grid(static_cast<int64_t>(sm_count()) * ctas_per_sm(kernel), p.groups, bpg);
+        constexpr auto kernel = nvfp4::quantize_grouped_kernel<FOUR, RULE, FQ>;
+        const dim3 grid = grouped_grid(static_cast<int64_t>(sm_count()) * ctas_per_sm<kernel>(), p.groups, bpg);
         kernel<<<grid, kThreads, 0, stream>>>(p);
     } else {
-        auto kernel = nvfp4::quantize_kernel<FOUR, RULE, FQ>;
-        const unsigned grid = grid_for(kernel, p.nblocks);
+        constexpr auto kernel = nvfp4::quantize_kernel<FOUR, RULE, FQ>;
+        const unsigned grid = grid_for<kernel>(p.nblocks);
         kernel<<<grid, kThreads, 0, stream>>>(p);
     }
     return launch_status();
@@ -153,8 +155,8 @@ nvfp4_status dispatch_quant(nvfp4_mode mode, nvfp4_rule rule, const nvfp4::Quant
 
 template <bool FOUR, int RULE>
 nvfp4_status launch_quant_gemm(const nvfp4::QuantParams& p, cudaStream_t stream) {
-    auto kernel = nvfp4::quantize_grouped_kernel<FOUR, RULE, false, true>;
-    kernel<<<grouped_grid(static_cast<int64_t>(sm_count()) * ctas_per_sm(kernel), 1, p.nblocks), kThreads, 0,
+    constexpr auto kernel = nvfp4::quantize_grouped_kernel<FOUR, RULE, false, true>;
+    kernel<<<grouped_grid(static_cast<int64_t>(sm_count()) * ctas_per_sm<kernel>(), 1, p.nblocks), kThreads, 0,
              stream>>>(p);
     return launch_status();
 }
@@ -197,7 +199,7 @@ nvfp4_status nvfp4_amax(const uint16_t* x, int64_t groups, int64_t rows, int64_t
         return NVFP4_ERR_CUDA;
     if (n == 0) return launch_status();
     const int64_t chunks = rows * cols / 16;
-    const int64_t full = static_cast<int64_t>(sm_count()) * ctas_per_sm(nvfp4::amax_kernel);
+    const int64_t full = static_cast<int64_t>(sm_count()) * ctas_per_sm<nvfp4::amax_kernel>();
     int64_t per_group = full / groups;
     if (per_group < 1) per_group = 1;
     const int64_t need = (chunks + kThreads - 1) / kThreads;
@@ -281,7 +283,7 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const
     p.nblocks = n / 16;
     p.groups = groups;
     p.gdiv = make_gdiv(groups, rows * cols / 16, p.nblocks);
-    const unsigned grid = grid_for(nvfp4::dequantize_kernel, (p.nblocks + 1) / 2);   // one pair per thread
+    const unsigned grid = grid_for<nvfp4::dequantize_kernel>((p.nblocks + 1) / 2);   // one pair per thread
     nvfp4::dequantize_kernel<<<grid, kThreads, 0, stream>>>(p);
     return launch_status();
 }
