@@ -64,8 +64,8 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
 
 // ---- quantize / fake-quant: CTAs inside one group at a time (scale table in shared memory) ------
 
-// Grid: x = CTAs per group, y = groups (looping when there are more than gridDim.y).
-// Each warp works on tiles of 64 consecutive blocks of its group: lane t quantizes blocks t and
+// Each warp works on tiles of 64 consecutive blocks of one group (the grid is described at
+// quantize_grouped_kernel): lane t quantizes blocks t and
 // t + 32 of the tile, so both 32-byte loads, both code stores and both scale stores of a warp
 // are contiguous, and each half-tile's 32 choice bits are one ballot word. The next tile's
 // blocks are loaded into registers before the current ones are worked on: in 4/6 mode into a
@@ -113,55 +113,79 @@ __device__ __forceinline__ void load_tile(const uint16_t* xg, uint32_t tile, uin
     ld32_stream(xg + static_cast<size_t>(min(a + 32u, last)) * 16, rb);
 }
 
+// Tiles tile, tile + stride, ... below tend of group g, with the group's scale table built
+// first (every thread of the CTA takes part: the table is shared). write_tscale: this CTA
+// stores the group's tensor scale.
+template <bool FOUR, int RULE, bool FQ, bool SWZ>
+__device__ __forceinline__ void quant_segment(const QuantParams& p, float2* tab, int64_t g, uint32_t tile,
+                                              uint32_t tend, uint32_t stride, uint32_t lane, bool write_tscale) {
+    constexpr float kSixM = FOUR ? 1536.0f : 2688.0f;   // 6 * 256 or 6 * 448
+    const uint32_t bpg = static_cast<uint32_t>(p.gdiv.bpg);
+    const int64_t base = g * static_cast<int64_t>(bpg);
+    const uint16_t* xg = p.x + base * 16;
+    uint32_t a0[8], a1[8];
+    if (tile < tend) load_tile(xg, tile, lane, bpg, a0, a1);   // in flight while the table is built
+    const GroupCtx gc = make_group<FOUR>(__ldg(p.amax + g), kSixM);
+    __syncthreads();                       // the previous group's table is no longer read
+    if (threadIdx.x < 128) tab[threadIdx.x] = scale_entry(threadIdx.x == 127 ? 126u : threadIdx.x, gc.alpha);
+    if (!FQ && write_tscale && threadIdx.x == 0) p.tscale[g] = gc.alpha;
+    __syncthreads();
+    uint8_t* cg = FQ ? nullptr : p.codes + base * 8;
+    uint8_t* sg = FQ ? nullptr : p.scales + base;
+    uint16_t* yg = FQ ? p.y + base * 16 : nullptr;
+    uint32_t* chw = reinterpret_cast<uint32_t*>(p.choice) + (base >> 5);   // base is a multiple of 32
+    if constexpr (!FOUR) {   // one prefetch buffer: two would not fit the 64-register budget
+        for (; tile < tend; tile += stride) {
+            uint32_t b0[8], b1[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                b0[k] = a0[k];
+                b1[k] = a1[k];
+            }
+            if (tile + stride < tend) load_tile(xg, tile + stride, lane, bpg, a0, a1);
+            quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, base, b0, b1);
+        }
+    } else {
+        uint32_t b0[8], b1[8];
+        while (tile < tend) {
+            uint32_t nt = tile + stride;
+            if (nt < tend) load_tile(xg, nt, lane, bpg, b0, b1);
+            quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, base, a0, a1);
+            tile = nt;
+            if (tile >= tend) break;
+            nt = tile + stride;
+            if (nt < tend) load_tile(xg, nt, lane, bpg, a0, a1);
+            quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, base, b0, b1);
+            tile = nt;
+        }
+    }
+}
+
+// One group: grid (x, 1), every warp of the grid strides over the group's tiles, so the warps
+// in flight read neighbouring tiles. Several groups: grid (x, 1), CTA b takes the contiguous
+// range [b T / x, (b + 1) T / x) of the T = groups * tiles_per_group tiles in group order, as
+// one segment per group it touches (its warps stride by the CTA's 8 warps inside a segment),
+// so every CTA slot works and the ranges differ by at most one tile.
 template <bool FOUR, int RULE, bool FQ, bool SWZ = false>
 __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kernel(const QuantParams p) {
-    constexpr float kSixM = FOUR ? 1536.0f : 2688.0f;   // 6 * 256 or 6 * 448
     __shared__ float2 tab[128];
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t bpg = static_cast<uint32_t>(p.gdiv.bpg);
     const uint32_t ntiles = (bpg + 63u) >> 6;
-    const uint32_t warps = gridDim.x * (kThreads / 32);
-    const uint32_t warp0 = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
-    for (int64_t g = blockIdx.y; g < p.groups; g += gridDim.y) {
-        const int64_t base = g * static_cast<int64_t>(bpg);
-        const uint16_t* xg = p.x + base * 16;
-        uint32_t tile = warp0;
-        uint32_t a0[8], a1[8];
-        if (tile < ntiles) load_tile(xg, tile, lane, bpg, a0, a1);   // in flight while the table is built
-        const GroupCtx gc = make_group<FOUR>(__ldg(p.amax + g), kSixM);
-        __syncthreads();                       // the previous group's table is no longer read
-        if (threadIdx.x < 128) tab[threadIdx.x] = scale_entry(threadIdx.x == 127 ? 126u : threadIdx.x, gc.alpha);
-        if (!FQ && blockIdx.x == 0 && threadIdx.x == 0) p.tscale[g] = gc.alpha;
-        __syncthreads();
-        uint8_t* cg = FQ ? nullptr : p.codes + base * 8;
-        uint8_t* sg = FQ ? nullptr : p.scales + base;
-        uint16_t* yg = FQ ? p.y + base * 16 : nullptr;
-        uint32_t* chw = reinterpret_cast<uint32_t*>(p.choice) + (base >> 5);   // base is a multiple of 32
-        if constexpr (!FOUR) {   // one prefetch buffer: two would not fit the 64-register budget
-            for (; tile < ntiles; tile += warps) {
-                uint32_t b0[8], b1[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    b0[k] = a0[k];
-                    b1[k] = a1[k];
-                }
-                if (tile + warps < ntiles) load_tile(xg, tile + warps, lane, bpg, a0, a1);
-                quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, base, b0, b1);
-            }
-        } else {
-            uint32_t b0[8], b1[8];
-            while (tile < ntiles) {
-                uint32_t nt = tile + warps;
-                if (nt < ntiles) load_tile(xg, nt, lane, bpg, b0, b1);
-                quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, base, a0, a1);
-                tile = nt;
-                if (tile >= ntiles) break;
-                nt = tile + warps;
-                if (nt < ntiles) load_tile(xg, nt, lane, bpg, a0, a1);
-                quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, base, b0, b1);
-                tile = nt;
-            }
-        }
+    constexpr uint32_t kWarps = kThreads / 32;
+    const uint32_t w = threadIdx.x >> 5;
+    // one call site for both layouts (the inlined tile loop is large; a second copy costs issue)
+    const bool one = p.groups == 1;
+    const int64_t total = p.groups * static_cast<int64_t>(ntiles);
+    const int64_t begin = one ? 0 : total * blockIdx.x / gridDim.x;
+    const int64_t end = one ? ntiles : total * (blockIdx.x + 1) / gridDim.x;
+    const uint32_t first = one ? blockIdx.x * kWarps + w : w, stride = one ? gridDim.x * kWarps : kWarps;
+    for (int64_t t = begin; t < end;) {
+        const int64_t g = t / ntiles;
+        const uint32_t t0 = static_cast<uint32_t>(t - g * ntiles);
+        const uint32_t t1 = static_cast<uint32_t>(min(end - g * ntiles, static_cast<int64_t>(ntiles)));
+        quant_segment<FOUR, RULE, FQ, SWZ>(p, tab, g, t0 + first, t1, stride, lane, one ? blockIdx.x == 0 : t0 == 0);
+        t = g * ntiles + t1;
     }
 }
 

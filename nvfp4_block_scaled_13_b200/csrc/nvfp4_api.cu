@@ -103,27 +103,15 @@ nvfp4_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
-// Grid of the grouped quantize kernel: gy rows of CTAs walk the groups (g = y, y + gy, ...),
-// gx CTAs share each group's warp tiles (64 blocks each). With `full` resident CTAs, pick the gy
-// that minimises the longest CTA's work, rounds x (tiles per warp + one tile's worth of
-// per-group setup), so that e.g. 64 experts on 296 CTA slots get 32 x 9 CTAs, not 64 x 4.
+// Grid of the grouped quantize kernel (one row of CTAs): one group takes enough CTAs for one
+// warp tile per warp, at most `full` (the resident CTAs); several groups take one CTA per
+// resident slot, at most one per warp tile of the whole tensor, and the kernel splits the
+// tiles of all groups into equal contiguous ranges.
 dim3 grouped_grid(int64_t full, int64_t groups, int64_t bpg) {
     constexpr int64_t kWarps = kThreads / 32;
     const int64_t ntiles = (bpg + 63) / 64;
-    const int64_t xmax = std::max<int64_t>(1, (ntiles + kWarps - 1) / kWarps);
-    const int64_t gymax = std::max<int64_t>(1, std::min<int64_t>(groups, std::min<int64_t>(full, 65535)));
-    int64_t best_gx = 1, best_gy = 1, best = INT64_MAX;
-    for (int64_t gy = 1; gy <= gymax; ++gy) {
-        const int64_t gx = std::max<int64_t>(1, std::min<int64_t>(full / gy, xmax));
-        const int64_t rounds = (groups + gy - 1) / gy;
-        const int64_t t = rounds * ((ntiles + gx * kWarps - 1) / (gx * kWarps) + 1);
-        if (t < best) {
-            best = t;
-            best_gx = gx;
-            best_gy = gy;
-        }
-    }
-    return dim3(static_cast<unsigned>(best_gx), static_cast<unsigned>(best_gy));
+    const int64_t want = groups == 1 ? (ntiles + kWarps - 1) / kWarps : groups * ntiles;
+    return dim3(static_cast<unsigned>(std::max<int64_t>(1, std::min(full, want))), 1u);
 }
 
 template <bool FOUR, int RULE, bool FQ>
