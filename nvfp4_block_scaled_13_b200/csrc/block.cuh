@@ -8,7 +8,8 @@
 // The quantizer is issue-bound, not memory-bound, so the per-block arithmetic is kept small:
 //  - block scales without a division: lo = RN(m * RN(RN(1/beta) (1 - 2^-20))) and
 //    hi = RN(m * RN(RN(1/beta) (1 + 2^-20))) bracket the exact quotient RN(m/beta), so when
-//    E4M3(lo) == E4M3(hi) the scale is proven; otherwise (rare) the exact division decides;
+//    E4M3(lo) == E4M3(hi) the scale is proven; otherwise the quotient sits at the E4M3
+//    rounding boundary between the two codes, and one exact fused multiply-add decides;
 //  - the decode scale d = RN(f32(s) * alpha) and its reciprocal for every E4M3 code s come
 //    from a 128-entry table per group in shared memory (kernels whose CTAs work inside one
 //    group at a time), or are computed per block (the generic kernel);
@@ -85,8 +86,8 @@ __device__ __forceinline__ float recip_clamped(float d) {
 
 // Per-group constants: alpha = amax / (6 M), beta_K = K * alpha, and the bracket factors
 // yl_K = RN(RN(1/beta_K) * (1 - 2^-20)), yh_K = RN(RN(1/beta_K) * (1 + 2^-20)) used to bracket
-// the block-scale quotients (valid when both betas lie in [2^-125, 2^125], so that every
-// factor is a normal number).
+// the block-scale quotients (`fast` when both betas lie in [2^-90, 2^125]: every factor is a
+// normal number, and the boundary test of block_scales is exact).
 struct GroupCtx {
     float alpha, beta6, beta4, yl6, yh6, yl4, yh4;
     bool fast;
@@ -99,7 +100,7 @@ __device__ __forceinline__ GroupCtx make_group(float amax, float six_m) {
     c.beta6 = __fmul_rn(6.0f, c.alpha);
     c.beta4 = __fmul_rn(4.0f, c.alpha);
     const float lo = FOUR ? c.beta4 : c.beta6;
-    c.fast = lo >= 0x1p-125f && c.beta6 <= 0x1p125f;
+    c.fast = lo >= 0x1p-90f && c.beta6 <= 0x1p125f;
     constexpr float kLo = 1.0f - 0x1p-20f, kHi = 1.0f + 0x1p-20f;
     const float y6 = c.fast ? __frcp_rn(c.beta6) : 0.0f, y4 = c.fast ? __frcp_rn(c.beta4) : 0.0f;
     c.yl6 = __fmul_rn(y6, kLo);
@@ -109,13 +110,34 @@ __device__ __forceinline__ GroupCtx make_group(float amax, float six_m) {
     return c;
 }
 
+// E4M3(RN(m / beta)) when the bracket gave adjacent codes s_lo < s_hi (the conversions of lo
+// and hi). The E4M3 rounding boundary M between them has at most 5 significant bits and
+// hi lies in [M, M (1 + 2^-19)], so M is hi truncated to 5 significant bits. With t =
+// RN(m / beta), u = the binary32 gap above M and M even in binary32:
+//   s_lo even (ties go down): s_hi iff t > M iff m / beta > M + u / 2,
+//   s_lo odd  (ties go up):   s_hi iff t >= M iff m / beta >= M - u / 2
+// (M is a power of two only between codes 0 and 1, where the smaller gap below M does not
+// matter). Multiplying by beta > 0 compares d = m - beta M with +-beta u / 2. Where
+// |m - beta M| <= 2^-18 m, beta M is a 29-bit multiple of 2^(e_beta + e_M - 27) >= 2^-149
+// (beta >= 2^-90, M >= 2^-10), so d needs at most 12 bits and the fused multiply-add is
+// exact; beta u / 2 = beta 2^(e_M - 24) is exact as well.
+__device__ __forceinline__ uint32_t scale_at_boundary(float m, float beta, float hi, uint32_t s_lo, uint32_t s_hi) {
+    const float mid = __uint_as_float(__float_as_uint(hi) & 0xFFF80000u);
+    const float d = __fmaf_rn(-beta, mid, m);
+    const float bu = __fmul_rn(beta, __uint_as_float((__float_as_uint(mid) & 0x7F800000u) - (24u << 23)));
+    return (s_lo & 1u) ? (d >= -bu ? s_hi : s_lo) : (d > bu ? s_hi : s_lo);
+}
+
 // E4M3(RN(m / beta_6)) in the low byte and E4M3(RN(m / beta_4)) in the high byte.
 // lo = RN(m * yl) and hi = RN(m * yh) carry three roundings of at most 2^-24 each on top of
 // the factors 1 -+ 2^-20, so lo < m/beta * (1 - 2^-21) < RN(m / beta) < hi whenever the
 // products are normal; below 2^-126 every one of them converts to E4M3 zero, and an overflow
 // saturates to 448 like the quotient it bounds. E4M3 rounding is monotone, so equal
-// conversions of lo and hi are the exact scale. Near a rounding boundary (about one block in
-// 2^15), or outside the factors' valid range, the exact division decides.
+// conversions of lo and hi are the exact scale; different ones are adjacent codes (E4M3
+// boundaries lie at least 2^-4 apart, relatively), and scale_at_boundary decides between
+// them. For data on a coarse grid, such as BF16 block maxima over a simple tensor scale,
+// RN(m / beta) falls exactly on an E4M3 boundary for a few percent of the blocks. Outside the
+// factors' valid range the exact division decides.
 template <bool FOUR>
 __device__ __forceinline__ uint32_t block_scales(float m, const GroupCtx& c) {
     if (c.fast) {
@@ -124,10 +146,15 @@ __device__ __forceinline__ uint32_t block_scales(float m, const GroupCtx& c) {
             const float2 hi = mul2(make_float2(m, m), make_float2(c.yh6, c.yh4));
             const uint32_t wl = e4m3x2(lo.x, lo.y), wh = e4m3x2(hi.x, hi.y);
             if (wl == wh) return wl;
+            uint32_t s6 = wl & 0xFFu, s4 = wl >> 8;
+            if (s6 != (wh & 0xFFu)) s6 = scale_at_boundary(m, c.beta6, hi.x, s6, wh & 0xFFu);
+            if (s4 != (wh >> 8)) s4 = scale_at_boundary(m, c.beta4, hi.y, s4, wh >> 8);
+            return s6 | (s4 << 8);
         } else {
             const float2 b = mul2(make_float2(m, m), make_float2(c.yl6, c.yh6));
             const uint32_t b6 = e4m3x2(b.x, b.y);
             if ((b6 & 0xFFu) == (b6 >> 8)) return b6 & 0xFFu;
+            return scale_at_boundary(m, c.beta6, b.y, b6 & 0xFFu, b6 >> 8);
         }
     }
     const float t6 = c.beta6 > 0.0f ? __fdiv_rn(m, c.beta6) : 0.0f;

@@ -181,3 +181,71 @@ def test_python_wrappers_round_trip(gpu):
     want = O.quantize(x, g, r, c, O.amax(x, g, r, c), 1, 2)
     U.assert_same("codes", q.codes.cpu().numpy(), want["codes"])
     U.assert_same("choice", q.choice.cpu().numpy(), want["choice"])
+
+
+# ---- block maxima whose scale quotient RN(m / beta) lies exactly on an E4M3 rounding boundary ----
+
+def _e4m3_boundaries() -> np.ndarray:
+    """Midpoints between consecutive non-negative E4M3 values (exact in binary32)."""
+    v = torch.arange(0, 127, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    return ((v[:-1] + v[1:]) / 2).astype(np.float32)
+
+
+def _boundary_groups(mode: int, n_groups: int):
+    """(amax, [(m, exact)]) for tensor maxima amax whose betas send some BF16 block maxima m
+    exactly onto an E4M3 boundary: m / beta equal to it (exact) or only rounded onto it."""
+    mids = _e4m3_boundaries()
+    ks = (6.0, 4.0) if mode == 1 else (6.0,)
+    bits = np.arange(0x3D00, 0x41F0, dtype=np.uint32)                 # BF16 amax in [0.031, 30)
+    found = []
+    for amax in (bits << 16).view(np.float32):
+        alpha = np.float32(O.tensor_scale(float(amax), mode))
+        hits = []
+        for k in ks:
+            beta = np.float32(np.float32(k) * alpha)
+            target = beta.astype(np.float64) * mids
+            for rnd in (np.floor, np.ceil):                             # the two BF16 neighbours
+                t = target.astype(np.float32).view(np.uint32).astype(np.int64)
+                hi16 = rnd(t / 65536.0).astype(np.int64)
+                m = (hi16.astype(np.uint32) << 16).view(np.float32)
+                ok = (m > 0) & (m < amax) & ((m / beta).astype(np.float32) == mids)
+                for mv, mid in zip(m[ok], mids[ok]):
+                    hits.append((np.float32(mv), bool(np.float64(mv) == np.float64(beta) * np.float64(mid))))
+        if hits:
+            hits.sort(key=lambda h: h[1])                                # rounded-onto ones first
+            found.append((np.float32(amax), hits))
+    # most hits first, keeping both kinds
+    found.sort(key=lambda f: -len(f[1]))
+    exact = [f for f in found if any(e for _, e in f[1])][: n_groups // 2]
+    rounded = [f for f in found if any(not e for _, e in f[1]) and f not in exact][: n_groups - len(exact)]
+    return exact + rounded
+
+
+def _boundary_tensor(groups, blocks_per_group: int, seed: int) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    out = []
+    for amax, hits in groups:
+        blocks = [np.concatenate([[amax], rng.uniform(-1, 1, 15) * amax * 0.9])]
+        for m, _ in hits[: blocks_per_group - 1]:
+            b = rng.uniform(-1, 1, 16) * m * 0.95
+            b[rng.integers(0, 16)] = m if rng.random() < 0.5 else -m
+            blocks.append(b)
+        while len(blocks) < blocks_per_group:
+            blocks.append(rng.standard_normal(16) * amax * 0.1)
+        out.append(np.concatenate(blocks))
+    return synth.to_bf16_bits(np.concatenate(out).astype(np.float32))
+
+
+@pytest.mark.parametrize("mode,rule", MODES, ids=MODE_IDS)
+def test_parity_scale_on_e4m3_boundary(gpu, mode, rule):
+    """Blocks whose scale quotient RN(m / beta) sits exactly on an E4M3 rounding boundary, where
+    the division-free bracket cannot decide and the boundary test or the tie-to-even rule
+    does: both the exact quotients and those rounded onto the boundary, each in its own
+    group's tensor scale, through the grouped kernel (64 blocks per group) and the flat one
+    (65)."""
+    groups = _boundary_groups(mode, 24)
+    for bpg in (64, 65):
+        used = [e for _, h in groups for _, e in h[: bpg - 1]]
+        assert sum(used) >= 100 and len(used) - sum(used) >= 20, (sum(used), len(used))
+        x = _boundary_tensor(groups, bpg, seed=bpg)
+        U.check_case(x, len(groups), bpg, 16, mode, rule)
