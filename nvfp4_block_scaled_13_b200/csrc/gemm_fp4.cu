@@ -13,15 +13,16 @@
 // One CTA computes a 128 x 256 tile of Y with warp-specialised roles over a 4-stage ring of
 // K slices (256 elements: four MMAs of K = 64) in shared memory:
 //   warp 0 (one lane)  TMA: B codes (and A codes when pre-quantized) as 128-byte swizzled
-//                      tiles, and the operands' 512-byte scale tiles as bulk copies, all
-//                      completing on the stage's "full" mbarrier;
+//                      tiles completing on the stage's "full" mbarrier, and the operands'
+//                      512-byte scale tiles as bulk copies completing on its "sffull" one
+//                      (on "full" as well in the prologue variant);
 //   warps 6-10         (prologue variant) quantize the stage's 128 x 256 BF16 activations
 //                      into the swizzled A tile and its scale tiles, then arrive on "full";
-//   last warps (lane 0; two, or one in the prologue variant) wait for "full", copy the
+//   last warps (lane 0; two, or one in the prologue variant) wait for "sffull", copy the
 //                      stage's scale tiles into tensor memory (tcgen05.cp.32x128b.warpx4, each
 //                      lane those of its share of the four MMAs) and commit the copies to the
 //                      stage's "sfready" mbarrier;
-//   warp 1 (one lane)  waits for "sfready", issues four
+//   warp 1 (one lane)  waits for "sfready" and "full", issues four
 //                      tcgen05.mma.kind::mxf4nvf4.block_scale.block16 into the FP32
 //                      accumulator in tensor memory, and commits them to the stage's "empty"
 //                      mbarrier, which releases the slot to the producers.
@@ -296,7 +297,8 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
                     const GemmParams p) {
     static_assert(!(QUANT && BF16), "the BF16 output is built for pre-quantized operands");
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full[kStages], empty[kStages], sfready[kStages], acc_full, acc_empty, drain;
+    __shared__ __align__(8) uint64_t full[kStages], empty[kStages], sfready[kStages], sffull[kStages], acc_full,
+        acc_empty, drain;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile uint32_t stop_sh;
     __shared__ float2 tab[128];
@@ -309,6 +311,10 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
     const int64_t ntn = (p.n + kBN - 1) / kBN, ntiles = ((p.m + kBM - 1) / kBM) * ntn;
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t full0 = smem_u32(&full[0]), empty0 = smem_u32(&empty[0]), sfr0 = smem_u32(&sfready[0]);
+    // pre-quantized operands: the slice's scale tiles complete on "sffull", its code tiles on
+    // "full", so the scale copies into tensor memory start while the codes still stream in; in
+    // the prologue variant the quantizer warps write the A scales, and everything uses "full"
+    const uint32_t sff0 = QUANT ? full0 : smem_u32(&sffull[0]);
     const uint32_t accf = smem_u32(&acc_full), acce = smem_u32(&acc_empty), drain_bar = smem_u32(&drain);
     constexpr int kSfWarp0 = gemm_threads<QUANT>() / 32 - sf_warps<QUANT>();   // first scale-copy warp
 
@@ -318,6 +324,7 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
             mbar_init(full0 + 8 * s, QUANT ? 1 + kQuantWarps : 1);
             mbar_init(empty0 + 8 * s, 1);
             mbar_init(sfr0 + 8 * s, sf_warps<QUANT>());
+            mbar_init(smem_u32(&sffull[s]), 1);
         }
         mbar_init(accf, 1);
         mbar_init(acce, epi_warps<QUANT>());
@@ -351,16 +358,21 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
                     const uint32_t fb = full0 + 8 * s, sA = sbase + s * kStageBytes, sB = sA + kABytes;
                     const uint32_t sSFA = sB + kBBytes, sSFB = sSFA + kSfaBytes;
                     const bool b_hi = (2 * tn + 1) * 128 < p.n;   // the tile's second 128 rows of B exist
-                    mbar_expect_tx(fb, (QUANT ? 0u : kABytes + kSfaBytes) + kBBytes + (b_hi ? kSfbBytes : kSfbBytes / 2));
-                    if (!QUANT) {
-                        tma_load_2d(sA, &tmap_a, ks * (kBK / 2), static_cast<int32_t>(tm * kBM), fb);
-                        bulk_load(sSFA, p.x_scales + (tm * n_ct + 4 * ks) * 512, kSfaBytes, fb);
+                    const uint32_t sb = sff0 + 8 * s;   // == fb in the prologue variant
+                    const uint32_t sf_bytes = (QUANT ? 0u : kSfaBytes) + (b_hi ? kSfbBytes : kSfbBytes / 2);
+                    if (QUANT) {
+                        mbar_expect_tx(fb, kBBytes + sf_bytes);
+                    } else {
+                        mbar_expect_tx(sb, sf_bytes);   // the small scale tiles first
+                        mbar_expect_tx(fb, kABytes + kBBytes);
+                        bulk_load(sSFA, p.x_scales + (tm * n_ct + 4 * ks) * 512, kSfaBytes, sb);
                     }
-                    tma_load_2d(sB, &tmap_b, ks * (kBK / 2), static_cast<int32_t>(tn * kBN), fb);
-                    bulk_load(sSFB, p.w_scales + (2 * tn * n_ct + 4 * ks) * 512, kSfbBytes / 2, fb);
+                    bulk_load(sSFB, p.w_scales + (2 * tn * n_ct + 4 * ks) * 512, kSfbBytes / 2, sb);
                     if (b_hi)
                         bulk_load(sSFB + kSfbBytes / 2, p.w_scales + ((2 * tn + 1) * n_ct + 4 * ks) * 512,
-                                  kSfbBytes / 2, fb);
+                                  kSfbBytes / 2, sb);
+                    if (!QUANT) tma_load_2d(sA, &tmap_a, ks * (kBK / 2), static_cast<int32_t>(tm * kBM), fb);
+                    tma_load_2d(sB, &tmap_b, ks * (kBK / 2), static_cast<int32_t>(tn * kBN), fb);
                 }
             }
         }
@@ -386,7 +398,8 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
                             break;
                         }
                     }
-                    if (!mbar_wait(sfr0 + 8 * s, phase)) {   // operands landed and scales copied
+                    if (!mbar_wait(sfr0 + 8 * s, phase) ||   // scales copied into tensor memory
+                        (!QUANT && !mbar_wait(full0 + 8 * s, phase))) {   // code tiles landed
                         ok = false;
                         break;
                     }
@@ -426,9 +439,9 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
 #pragma unroll
                 for (int s = 0; s < kStages; ++s) {
                     if (gg >= total) break;
-                    // slice gg's "full" completes only after the MMAs that last read this slot's
+                    // slice gg's scale tiles land only after the MMAs that last read this slot's
                     // scale columns have finished (the producer refilled the slot after "empty")
-                    if (!mbar_wait(full0 + 8 * s, phase)) {
+                    if (!mbar_wait(sff0 + 8 * s, phase)) {
                         ok = false;
                         break;
                     }
