@@ -148,6 +148,41 @@ NVFP4_API nvfp4_status nvfp4_fakequant(const uint16_t* x, int64_t groups, int64_
                              const float* amax, nvfp4_mode mode, nvfp4_rule rule,
                              uint16_t* y, uint8_t* choice, cudaStream_t stream);
 
+/* Bit set in a quantizer's status word when the grid-wide wait of nvfp4_amax_quantize or
+ * nvfp4_amax_fakequant timed out (about two seconds); the outputs other than amax are then
+ * not written. */
+#define NVFP4_QUANT_TIMEOUT 2u
+
+/* nvfp4_amax followed by nvfp4_quantize in one launch: the dynamic tensor scale with the
+ * fused amax ([FOS] Implementation details: the FP32 tensor scale comes from the tensor's
+ * absolute maximum). Every CTA reduces max |x| over exactly the tiles it then quantizes,
+ * all CTAs meet at a grid-wide barrier (a cooperative launch keeps them resident), and the
+ * quantization re-reads the tiles, from L2 when the tensor fits there (126 MB). Outputs are
+ * bit-identical to the two calls.
+ *   x, groups, rows, cols, mode, rule, codes, scales, tscale, choice as nvfp4_quantize (in/out)
+ *   amax       [groups] float, 4-byte aligned: max |x| per group, written here          (out)
+ *   workspace  NULL, or one 4-byte-aligned device word the call may use (zero-filled in
+ *              stream order before the launch). With NULL the call uses one word of
+ *              library memory per device and allocates nothing; such calls must not run
+ *              concurrently on one device (different streams), while calls with their own
+ *              workspaces may.                                                    (scratch)
+ *   status     NULL, or a device word; NVFP4_QUANT_TIMEOUT is or-ed in on a timed-out
+ *              grid-wide wait                                                        (in/out)
+ * Group layouts the grouped quantizer does not take (several groups whose block count is not
+ * a multiple of 32), and empty tensors, run as the two separate launches. Errors as
+ * nvfp4_quantize, plus NVFP4_ERR_CUDA when the cooperative launch is refused. */
+NVFP4_API nvfp4_status nvfp4_amax_quantize(const uint16_t* x, int64_t groups, int64_t rows, int64_t cols,
+                                           nvfp4_mode mode, nvfp4_rule rule, float* amax, uint8_t* codes,
+                                           uint8_t* scales, float* tscale, uint8_t* choice, uint32_t* workspace,
+                                           uint32_t* status, cudaStream_t stream);
+
+/* nvfp4_amax followed by nvfp4_fakequant in one launch, as nvfp4_amax_quantize.
+ *   y  [groups, rows, cols] BF16 bits, 32-byte aligned                                  (out) */
+NVFP4_API nvfp4_status nvfp4_amax_fakequant(const uint16_t* x, int64_t groups, int64_t rows, int64_t cols,
+                                            nvfp4_mode mode, nvfp4_rule rule, float* amax, uint16_t* y,
+                                            uint8_t* choice, uint32_t* workspace, uint32_t* status,
+                                            cudaStream_t stream);
+
 /* Quantize a [rows, cols] BF16 matrix for a Blackwell block-scaled FP4 tensor-core GEMM, in
  * which it is the K-major operand (cols = K). NVFP4 weights and activations are run on
  * Blackwell's native FP4 tensor cores ("NVIDIA Model Optimizerを用いたNemotron 3.5 Lightning

@@ -20,15 +20,17 @@ import os
 from typing import NamedTuple
 
 __all__ = [
-    "load", "library_path", "Nvfp4Error",
+    "load", "library_path", "Nvfp4Error", "Nvfp4TimeoutError",
     "SCALE6", "FOUR_OVER_SIX", "RULE_MAXERR", "RULE_MAE", "RULE_MSE",
-    "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_quantize_gemm", "nvfp4_qad_kl",
+    "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_amax_quantize",
+    "nvfp4_amax_fakequant", "QUANT_TIMEOUT", "nvfp4_quantize_gemm", "nvfp4_qad_kl",
     "nvfp4_gemm", "nvfp4_gemm_bf16", "nvfp4_gemm_quantize_x", "GEMM_TIMEOUT", "nvfp4_status_string", "nvfp4_version",
-    "Quantized", "amax", "quantize", "fakequant", "dequantize", "quantize_for_gemm", "gemm_scale_bytes",
+    "Quantized", "amax", "quantize", "fakequant", "dequantize", "amax_quantize", "amax_fakequant", "quantize_for_gemm", "gemm_scale_bytes",
     "qad_kl", "fakequant_ste", "gemm", "gemm_bf16", "gemm_quantize_x",
 ]
 
 GEMM_TIMEOUT = 1   # bit of a GEMM's status word: a bounded wait for the tensor core timed out
+QUANT_TIMEOUT = 2  # bit of a quantizer's status word: the grid-wide wait of a one-launch amax timed out
 
 SCALE6, FOUR_OVER_SIX = 0, 1
 RULE_MAXERR, RULE_MAE, RULE_MSE = 0, 1, 2
@@ -44,6 +46,10 @@ class Nvfp4Error(RuntimeError):
     def __init__(self, status: int, func: str):
         self.status = status
         super().__init__(f"{func}: {nvfp4_status_string(status)} (status {status})")
+
+
+class Nvfp4TimeoutError(RuntimeError):
+    """A kernel's bounded wait timed out, as its status word reports (its outputs are partial)."""
 
 
 def library_path() -> str:
@@ -67,9 +73,12 @@ def load():
         L.nvfp4_qad_kl.argtypes = [vp, vp, i64, i64, ctypes.c_float, ctypes.c_float, vp, vp, vp]
         L.nvfp4_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp]
         L.nvfp4_gemm_bf16.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp]
+        L.nvfp4_amax_quantize.argtypes = [vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.nvfp4_amax_fakequant.argtypes = [vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp]
         L.nvfp4_gemm_quantize_x.argtypes = [vp, vp, i32, i32, vp, vp, vp, i64, i64, i64, vp, vp, vp]
         for f in (L.nvfp4_amax, L.nvfp4_quantize, L.nvfp4_dequantize, L.nvfp4_fakequant, L.nvfp4_quantize_gemm,
-                  L.nvfp4_qad_kl, L.nvfp4_gemm, L.nvfp4_gemm_bf16, L.nvfp4_gemm_quantize_x):
+                  L.nvfp4_qad_kl, L.nvfp4_gemm, L.nvfp4_gemm_bf16, L.nvfp4_gemm_quantize_x, L.nvfp4_amax_quantize,
+                  L.nvfp4_amax_fakequant):
             f.restype = i32
         L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
         L.nvfp4_version.argtypes, L.nvfp4_version.restype = [], i32
@@ -135,6 +144,20 @@ def nvfp4_dequantize(codes, scales, tscale, groups, rows, cols, y, stream=None):
 def nvfp4_fakequant(x, groups, rows, cols, amax, mode, rule, y, choice=None, stream=None):
     _check(load().nvfp4_fakequant(_ptr(x), groups, rows, cols, _ptr(amax), _mode(mode), _rule(rule),
                                   _ptr(y), _ptr(choice), _stream(stream)), "nvfp4_fakequant")
+
+
+def nvfp4_amax_quantize(x, groups, rows, cols, mode, rule, amax, codes, scales, tscale, choice=None, workspace=None,
+                        status=None, stream=None):
+    _check(load().nvfp4_amax_quantize(_ptr(x), groups, rows, cols, _mode(mode), _rule(rule), _ptr(amax), _ptr(codes),
+                                      _ptr(scales), _ptr(tscale), _ptr(choice), _ptr(workspace), _ptr(status),
+                                      _stream(stream)), "nvfp4_amax_quantize")
+
+
+def nvfp4_amax_fakequant(x, groups, rows, cols, mode, rule, amax, y, choice=None, workspace=None, status=None,
+                         stream=None):
+    _check(load().nvfp4_amax_fakequant(_ptr(x), groups, rows, cols, _mode(mode), _rule(rule), _ptr(amax), _ptr(y),
+                                       _ptr(choice), _ptr(workspace), _ptr(status), _stream(stream)),
+           "nvfp4_amax_fakequant")
 
 
 def nvfp4_gemm(x_codes, x_scales, x_tscale, w_codes, w_scales, w_tscale, m, n, k, y, status=None, stream=None):
@@ -246,6 +269,43 @@ def fakequant(x, mode="four_over_six", rule="mse", groups: int = 1, amax_values=
     return out
 
 
+def amax_quantize(x, mode="four_over_six", rule="mse", groups: int = 1, with_choice=True, stream=None):
+    """(Quantized, amax): the tensor amax and the quantization in one launch. Raises if the
+    launch's grid-wide wait timed out."""
+    import torch
+
+    g, r, c = _shape3(x, groups)
+    n = g * r * c
+    nb = n // 16
+    dev = x.device
+    amax_out = torch.empty(g, dtype=torch.float32, device=dev)
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(nb, dtype=torch.uint8, device=dev)
+    tscale = torch.empty(g, dtype=torch.float32, device=dev)
+    choice = torch.empty(max(1, (nb + 7) // 8), dtype=torch.uint8, device=dev) if with_choice else None
+    work = torch.empty(2, dtype=torch.int32, device=dev)   # [0] barrier counter, [1] status
+    work[1:].zero_()
+    nvfp4_amax_quantize(x, g, r, c, mode, rule, amax_out, codes, scales, tscale, choice, work[0:1], work[1:2], stream)
+    if int(work[1].item()) & QUANT_TIMEOUT:
+        raise Nvfp4TimeoutError("nvfp4_amax_quantize: the grid-wide wait timed out")
+    return Quantized(codes, scales, tscale, choice, (g, r, c)), amax_out
+
+
+def amax_fakequant(x, mode="four_over_six", rule="mse", groups: int = 1, out=None, choice=None, stream=None):
+    """(fake-quantized BF16, amax) in one launch."""
+    import torch
+
+    g, r, c = _shape3(x, groups)
+    amax_out = torch.empty(g, dtype=torch.float32, device=x.device)
+    if out is None:
+        out = torch.empty_like(x, dtype=torch.bfloat16)
+    work = torch.zeros(2, dtype=torch.int32, device=x.device)
+    nvfp4_amax_fakequant(x, g, r, c, mode, rule, amax_out, out, choice, work[0:1], work[1:2], stream)
+    if int(work[1].item()) & QUANT_TIMEOUT:
+        raise Nvfp4TimeoutError("nvfp4_amax_fakequant: the grid-wide wait timed out")
+    return out, amax_out
+
+
 def gemm_scale_bytes(rows: int, cols: int) -> int:
     """Size of the tiled scale buffer of nvfp4_quantize_gemm: roundup(rows, 128) * roundup(cols / 16, 4)."""
     return (rows + 127) // 128 * 128 * ((cols // 16 + 3) // 4 * 4)
@@ -282,7 +342,7 @@ def gemm(xq, wq, stream=None):
     status = torch.zeros(1, dtype=torch.int32, device=xc.device)
     nvfp4_gemm(xc, xs, xt, wc, ws, wt, m, n, k, y, status, stream)
     if int(status.item()) & GEMM_TIMEOUT:
-        raise Nvfp4Error("nvfp4_gemm: a wait for the tensor core timed out")
+        raise Nvfp4TimeoutError("nvfp4_gemm: a wait for the tensor core timed out")
     return y
 
 
@@ -298,7 +358,7 @@ def gemm_bf16(xq, wq, stream=None):
     status = torch.zeros(1, dtype=torch.int32, device=xc.device)
     nvfp4_gemm_bf16(xc, xs, xt, wc, ws, wt, m, n, k, y, y_amax, status, stream)
     if int(status.item()) & GEMM_TIMEOUT:
-        raise Nvfp4Error("nvfp4_gemm_bf16: a wait for the tensor core timed out")
+        raise Nvfp4TimeoutError("nvfp4_gemm_bf16: a wait for the tensor core timed out")
     return y, y_amax
 
 
@@ -315,7 +375,7 @@ def gemm_quantize_x(x, wq, mode="four_over_six", rule="mse", amax_values=None, s
     status = torch.zeros(1, dtype=torch.int32, device=x.device)
     nvfp4_gemm_quantize_x(x, amax_values, mode, rule, wc, ws, wt, m, n, k, y, status, stream)
     if int(status.item()) & GEMM_TIMEOUT:
-        raise Nvfp4Error("nvfp4_gemm_quantize_x: a wait for the tensor core timed out")
+        raise Nvfp4TimeoutError("nvfp4_gemm_quantize_x: a wait for the tensor core timed out")
     return y
 
 

@@ -116,7 +116,9 @@ __device__ __forceinline__ void load_tile(const uint16_t* xg, uint32_t tile, uin
 // Tiles tile, tile + stride, ... below tend of group g, with the group's scale table built
 // first (every thread of the CTA takes part: the table is shared). write_tscale: this CTA
 // stores the group's tensor scale.
-template <bool FOUR, int RULE, bool FQ, bool SWZ>
+// FRESH: the amax was written during this launch (by other CTAs), so it is read with a
+// gpu-scope acquire load rather than through the read-only cache.
+template <bool FOUR, int RULE, bool FQ, bool SWZ, bool FRESH = false>
 __device__ __forceinline__ void quant_segment(const QuantParams& p, float2* tab, int64_t g, uint32_t tile,
                                               uint32_t tend, uint32_t stride, uint32_t lane, bool write_tscale) {
     constexpr float kSixM = FOUR ? 1536.0f : 2688.0f;   // 6 * 256 or 6 * 448
@@ -125,7 +127,7 @@ __device__ __forceinline__ void quant_segment(const QuantParams& p, float2* tab,
     const uint16_t* xg = p.x + base * 16;
     uint32_t a0[8], a1[8];
     if (tile < tend) load_tile(xg, tile, lane, bpg, a0, a1);   // in flight while the table is built
-    const GroupCtx gc = make_group<FOUR>(__ldg(p.amax + g), kSixM);
+    const GroupCtx gc = make_group<FOUR>(FRESH ? ld_acquire_f32(p.amax + g) : __ldg(p.amax + g), kSixM);
     __syncthreads();                       // the previous group's table is no longer read
     if (threadIdx.x < 128) tab[threadIdx.x] = scale_entry(threadIdx.x == 127 ? 126u : threadIdx.x, gc.alpha);
     if (!FQ && write_tscale && threadIdx.x == 0) p.tscale[g] = gc.alpha;
@@ -185,6 +187,99 @@ __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kerne
         const uint32_t t0 = static_cast<uint32_t>(t - g * ntiles);
         const uint32_t t1 = static_cast<uint32_t>(min(end - g * ntiles, static_cast<int64_t>(ntiles)));
         quant_segment<FOUR, RULE, FQ, SWZ>(p, tab, g, t0 + first, t1, stride, lane, one ? blockIdx.x == 0 : t0 == 0);
+        t = g * ntiles + t1;
+    }
+}
+
+// ---- amax and quantize / fake-quant in one launch (a grid-wide wait between them) -------------
+
+// Max |x| (as BF16 magnitude bits, packed pairs) over the lane's blocks of tiles tile, tile +
+// stride, ... below tend of one group (the tiles the same lane quantizes afterwards).
+__device__ __forceinline__ uint32_t segment_max2(const uint16_t* xg, uint32_t tile, uint32_t tend, uint32_t stride,
+                                                 uint32_t lane, uint32_t bpg) {
+    uint32_t m2 = 0;
+    for (; tile < tend; tile += stride) {
+        uint32_t a[8], b[8];
+        load_tile(xg, tile, lane, bpg, a, b);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            asm("max.u16x2 %0, %0, %1;" : "+r"(m2) : "r"(a[k] & 0x7FFF7FFFu));
+            asm("max.u16x2 %0, %0, %1;" : "+r"(m2) : "r"(b[k] & 0x7FFF7FFFu));
+        }
+    }
+    return m2;
+}
+
+// Maximum over the CTA of one value per thread, combined into *out with an unsigned atomic
+// maximum (binary32 values >= 0 order like their bits). Every thread of the CTA calls it.
+__device__ __forceinline__ void cta_max_to(uint32_t* red, uint32_t v, float* out) {
+    v = __reduce_max_sync(0xFFFFFFFFu, v);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t w = lane < kThreads / 32 ? red[lane] : 0u;
+        w = __reduce_max_sync(0xFFFFFFFFu, w);
+        if (lane == 0 && w != 0) atomicMax(reinterpret_cast<unsigned int*>(out), w << 16);
+    }
+    __syncthreads();
+}
+
+// Quantize (or fake-quantize) with the group amaxes found in the same launch: every CTA first
+// reduces max |x| over exactly the tiles it quantizes afterwards into p.amax (zero-filled
+// before the launch), then all CTAs meet at a grid-wide barrier on *arrive (zero-filled
+// before the launch), then they quantize as quantize_grouped_kernel does, re-reading their
+// tiles (from L2 when the tensor fits there). The grid must be co-resident (a cooperative
+// launch). The barrier's wait is bounded (about two seconds): on timeout the kernel or-s
+// NVFP4_QUANT_TIMEOUT into *status (nullable) and quantizes nothing.
+template <bool FOUR, int RULE, bool FQ>
+__global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_amax_kernel(const QuantParams p, uint32_t* arrive,
+                                                                                uint32_t* status) {
+    __shared__ float2 tab[128];
+    __shared__ uint32_t red[kThreads / 32];
+    __shared__ uint32_t go;
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t bpg = static_cast<uint32_t>(p.gdiv.bpg);
+    const uint32_t ntiles = (bpg + 63u) >> 6;
+    constexpr uint32_t kWarps = kThreads / 32;
+    const uint32_t w = threadIdx.x >> 5;
+    const bool one = p.groups == 1;
+    const int64_t total = p.groups * static_cast<int64_t>(ntiles);
+    const int64_t begin = one ? 0 : total * blockIdx.x / gridDim.x;
+    const int64_t end = one ? ntiles : total * (blockIdx.x + 1) / gridDim.x;
+    const uint32_t first = one ? blockIdx.x * kWarps + w : w, stride = one ? gridDim.x * kWarps : kWarps;
+    float* amax = const_cast<float*>(p.amax);
+    for (int64_t t = begin; t < end;) {   // phase 1: this CTA's share of every group's amax
+        const int64_t g = t / ntiles;
+        const uint32_t t0 = static_cast<uint32_t>(t - g * ntiles);
+        const uint32_t t1 = static_cast<uint32_t>(min(end - g * ntiles, static_cast<int64_t>(ntiles)));
+        const uint32_t m2 = segment_max2(p.x + g * static_cast<int64_t>(bpg) * 16, t0 + first, t1, stride, lane, bpg);
+        cta_max_to(red, max(m2 & 0xFFFFu, m2 >> 16), amax + g);
+        t = g * ntiles + t1;
+    }
+    if (threadIdx.x == 0) {   // grid-wide barrier: release this CTA's maxima, wait for every CTA
+        __threadfence();
+        atomicAdd(arrive, 1u);
+        uint32_t ok = 1;
+        const unsigned long long t0 = clock64();
+        while (ld_acquire_u32(arrive) < gridDim.x) {
+            if (clock64() - t0 > 4000000000ull) {
+                ok = 0;
+                if (status != nullptr) atomicOr(status, NVFP4_QUANT_TIMEOUT);
+                break;
+            }
+            __nanosleep(64);
+        }
+        go = ok;
+    }
+    __syncthreads();
+    if (!go) return;
+    for (int64_t t = begin; t < end;) {   // phase 2: quantize with the finished amaxes
+        const int64_t g = t / ntiles;
+        const uint32_t t0 = static_cast<uint32_t>(t - g * ntiles);
+        const uint32_t t1 = static_cast<uint32_t>(min(end - g * ntiles, static_cast<int64_t>(ntiles)));
+        quant_segment<FOUR, RULE, FQ, false, true>(p, tab, g, t0 + first, t1, stride, lane,
+                                                   one ? blockIdx.x == 0 : t0 == 0);
         t = g * ntiles + t1;
     }
 }

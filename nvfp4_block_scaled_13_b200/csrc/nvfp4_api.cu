@@ -141,6 +141,35 @@ nvfp4_status dispatch_quant(nvfp4_mode mode, nvfp4_rule rule, const nvfp4::Quant
     }
 }
 
+// Barrier counter of nvfp4_amax_quantize / nvfp4_amax_fakequant calls without a workspace:
+// library memory (one per device), so those calls allocate nothing; they must not overlap.
+__device__ __align__(256) uint32_t g_amax_quant_scratch[64];
+
+template <bool FOUR, int RULE, bool FQ>
+nvfp4_status launch_quant_amax(const nvfp4::QuantParams& p, uint32_t* arrive, uint32_t* status, cudaStream_t stream) {
+    constexpr auto kernel = nvfp4::quantize_amax_kernel<FOUR, RULE, FQ>;
+    // every CTA must be resident for the grid-wide barrier: a cooperative launch of at most
+    // the resident CTAs (it fails instead of hanging if they do not fit)
+    const dim3 grid = grouped_grid(static_cast<int64_t>(sm_count()) * ctas_per_sm<kernel>(), p.groups, p.gdiv.bpg);
+    nvfp4::QuantParams pp = p;
+    void* args[] = {&pp, &arrive, &status};
+    if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), grid, dim3(kThreads), args, 0, stream) !=
+        cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return launch_status();
+}
+
+template <bool FQ>
+nvfp4_status dispatch_quant_amax(nvfp4_mode mode, nvfp4_rule rule, const nvfp4::QuantParams& p, uint32_t* arrive,
+                                 uint32_t* status, cudaStream_t s) {
+    if (mode == NVFP4_SCALE6) return launch_quant_amax<false, nvfp4::kMse, FQ>(p, arrive, status, s);
+    switch (rule) {
+        case NVFP4_RULE_MAXERR: return launch_quant_amax<true, nvfp4::kMaxErr, FQ>(p, arrive, status, s);
+        case NVFP4_RULE_MAE: return launch_quant_amax<true, nvfp4::kMae, FQ>(p, arrive, status, s);
+        default: return launch_quant_amax<true, nvfp4::kMse, FQ>(p, arrive, status, s);
+    }
+}
+
 template <bool FOUR, int RULE>
 nvfp4_status launch_quant_gemm(const nvfp4::QuantParams& p, cudaStream_t stream) {
     constexpr auto kernel = nvfp4::quantize_grouped_kernel<FOUR, RULE, false, true>;
@@ -169,6 +198,52 @@ nvfp4_status check_mode_rule(nvfp4_mode mode, nvfp4_rule rule) {
 __global__ void tensor_scale_only_kernel(const float* amax, float* tscale, int64_t groups, float six_m) {
     for (int64_t g = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; g < groups; g += int64_t(gridDim.x) * blockDim.x)
         tscale[g] = __fdiv_rn(amax[g], six_m);
+}
+
+// nvfp4_amax_quantize (y == nullptr) and nvfp4_amax_fakequant (y != nullptr).
+nvfp4_status amax_quant_impl(const uint16_t* x, int64_t groups, int64_t rows, int64_t cols, nvfp4_mode mode,
+                             nvfp4_rule rule, float* amax, uint8_t* codes, uint8_t* scales, float* tscale,
+                             uint16_t* y, uint8_t* choice, uint32_t* workspace, uint32_t* status, cudaStream_t stream) {
+    const bool fq = y != nullptr;
+    if (amax == nullptr || (!fq && tscale == nullptr)) return NVFP4_ERR_NULL;
+    int64_t n = 0;
+    nvfp4_status st = check_shape(groups, rows, cols, &n);
+    if (st != NVFP4_OK) return st;
+    if (n > 0 && (x == nullptr || (!fq && (codes == nullptr || scales == nullptr)))) return NVFP4_ERR_NULL;
+    st = check_mode_rule(mode, rule);
+    if (st != NVFP4_OK) return st;
+    if (!aligned(amax, 4) || (tscale && !aligned(tscale, 4)) || (choice && !aligned(choice, 4)) ||
+        (workspace && !aligned(workspace, 4)) || (status && !aligned(status, 4)))
+        return NVFP4_ERR_ALIGN;
+    if (n > 0 && (!aligned(x, 32) || (!fq && !aligned(codes, 8)) || (fq && !aligned(y, 32)))) return NVFP4_ERR_ALIGN;
+    const int64_t bpg = rows * cols / 16;
+    if (n == 0 || !((groups == 1 || bpg % 32 == 0) && bpg < (int64_t(1) << 30))) {
+        // empty tensors and group layouts the one-launch kernel does not take: the two passes
+        st = nvfp4_amax(x, groups, rows, cols, amax, stream);
+        if (st != NVFP4_OK) return st;
+        return fq ? nvfp4_fakequant(x, groups, rows, cols, amax, mode, rule, y, choice, stream)
+                  : nvfp4_quantize(x, groups, rows, cols, amax, mode, rule, codes, scales, tscale, choice, stream);
+    }
+    if (workspace == nullptr &&
+        cudaGetSymbolAddress(reinterpret_cast<void**>(&workspace), g_amax_quant_scratch) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    if (cudaMemsetAsync(amax, 0, static_cast<size_t>(groups) * sizeof(float), stream) != cudaSuccess ||
+        cudaMemsetAsync(workspace, 0, sizeof(uint32_t), stream) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    nvfp4::QuantParams p{};
+    p.x = x;
+    p.amax = amax;
+    p.codes = fq ? nullptr : codes;
+    p.scales = fq ? nullptr : scales;
+    p.tscale = fq ? nullptr : tscale;
+    p.choice = choice;
+    p.y = y;
+    p.nblocks = n / 16;
+    p.choice_bytes = (p.nblocks + 7) / 8;
+    p.groups = groups;
+    p.gdiv = make_gdiv(groups, bpg, p.nblocks);
+    return fq ? dispatch_quant_amax<true>(mode, rule, p, workspace, status, stream)
+              : dispatch_quant_amax<false>(mode, rule, p, workspace, status, stream);
 }
 
 }  // namespace
@@ -253,6 +328,28 @@ nvfp4_status nvfp4_fakequant(const uint16_t* x, int64_t groups, int64_t rows, in
     p.groups = groups;
     p.gdiv = make_gdiv(groups, rows * cols / 16, p.nblocks);
     return dispatch_quant<true>(mode, rule, p, stream);
+}
+
+nvfp4_status nvfp4_amax_quantize(const uint16_t* x, int64_t groups, int64_t rows, int64_t cols, nvfp4_mode mode,
+                                 nvfp4_rule rule, float* amax, uint8_t* codes, uint8_t* scales, float* tscale,
+                                 uint8_t* choice, uint32_t* workspace, uint32_t* status, cudaStream_t stream) {
+    return amax_quant_impl(x, groups, rows, cols, mode, rule, amax, codes, scales, tscale, nullptr, choice, workspace,
+                           status, stream);
+}
+
+nvfp4_status nvfp4_amax_fakequant(const uint16_t* x, int64_t groups, int64_t rows, int64_t cols, nvfp4_mode mode,
+                                  nvfp4_rule rule, float* amax, uint16_t* y, uint8_t* choice, uint32_t* workspace,
+                                  uint32_t* status, cudaStream_t stream) {
+    if (y == nullptr) {   // y selects the fake-quant variant inside; check it here
+        int64_t n = 0;
+        const nvfp4_status st = check_shape(groups, rows, cols, &n);
+        if (st != NVFP4_OK) return st;
+        if (n > 0) return NVFP4_ERR_NULL;
+        if (amax == nullptr) return NVFP4_ERR_NULL;
+        return nvfp4_amax(x, groups, rows, cols, amax, stream);
+    }
+    return amax_quant_impl(x, groups, rows, cols, mode, rule, amax, nullptr, nullptr, nullptr, y, choice, workspace,
+                           status, stream);
 }
 
 nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tscale, int64_t groups,

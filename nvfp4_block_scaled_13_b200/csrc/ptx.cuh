@@ -86,6 +86,17 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
     return d;
 }
 
+// gpu-scope acquire loads (values written by other CTAs of the same launch)
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ float ld_acquire_f32(const float* p) {
+    return __uint_as_float(ld_acquire_u32(reinterpret_cast<const uint32_t*>(p)));
+}
+
 // ---- format conversions ------------------------------------------------------------------
 
 // Eight binary32 values (four pairs p[j] = (element 2j, element 2j+1)) -> eight E2M1 codes

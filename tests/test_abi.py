@@ -19,7 +19,7 @@ def header_functions(path):
 
 def test_header_declares_the_boundary():
     names = header_functions(os.path.join(ROOT, "include", "nvfp4.h"))
-    assert names == ["nvfp4_amax", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_gemm", "nvfp4_gemm_bf16", "nvfp4_gemm_quantize_x",
+    assert names == ["nvfp4_amax", "nvfp4_amax_fakequant", "nvfp4_amax_quantize", "nvfp4_dequantize", "nvfp4_fakequant", "nvfp4_gemm", "nvfp4_gemm_bf16", "nvfp4_gemm_quantize_x",
                      "nvfp4_qad_kl", "nvfp4_quantize", "nvfp4_quantize_gemm", "nvfp4_status_string",
                      "nvfp4_version"]
 
@@ -114,6 +114,23 @@ A = 1 << 20          # 32-byte aligned
     (lambda L: L.nvfp4_gemm_quantize_x(None, A, 1, 2, A, A, A, 128, 256, 256, A, None, None), 1),
     (lambda L: L.nvfp4_gemm_quantize_x(A, None, 1, 2, A, A, A, 128, 256, 256, A, None, None), 1),
     (lambda L: L.nvfp4_gemm_quantize_x(A + 16, A, 1, 2, A, A, A, 128, 256, 256, A, None, None), 3),
+    # nvfp4_amax_quantize(x, G, R, C, mode, rule, amax, codes, scales, tscale, choice, workspace, status, stream)
+    (lambda L: L.nvfp4_amax_quantize(A, 1, 4, 32, 1, 2, None, A, A, A, None, None, None, None), 1),
+    (lambda L: L.nvfp4_amax_quantize(A, 1, 4, 32, 1, 2, A, None, A, A, None, None, None, None), 1),
+    (lambda L: L.nvfp4_amax_quantize(A, 1, 4, 32, 1, 2, A, A, A, None, None, None, None, None), 1),
+    (lambda L: L.nvfp4_amax_quantize(A, 1, 4, 33, 1, 2, A, A, A, A, None, None, None, None), 2),
+    (lambda L: L.nvfp4_amax_quantize(A, 1, 4, 32, 3, 2, A, A, A, A, None, None, None, None), 4),
+    (lambda L: L.nvfp4_amax_quantize(A, 1, 4, 32, 1, 3, A, A, A, A, None, None, None, None), 5),
+    (lambda L: L.nvfp4_amax_quantize(A + 2, 1, 4, 32, 1, 2, A, A, A, A, None, None, None, None), 3),
+    (lambda L: L.nvfp4_amax_quantize(A, 1, 4, 32, 1, 2, A + 2, A, A, A, None, None, None, None), 3),
+    (lambda L: L.nvfp4_amax_quantize(A, 1, 4, 32, 1, 2, A, A, A, A, None, A + 2, None, None), 3),
+    (lambda L: L.nvfp4_amax_quantize(A, 1, 4, 32, 1, 2, A, A, A, A, None, None, A + 1, None), 3),
+    # nvfp4_amax_fakequant(x, G, R, C, mode, rule, amax, y, choice, workspace, status, stream)
+    (lambda L: L.nvfp4_amax_fakequant(A, 1, 4, 32, 1, 2, None, A, None, None, None, None), 1),
+    (lambda L: L.nvfp4_amax_fakequant(A, 1, 4, 32, 1, 2, A, None, None, None, None, None), 1),
+    (lambda L: L.nvfp4_amax_fakequant(A, 1, 4, 31, 1, 2, A, A, None, None, None, None), 2),
+    (lambda L: L.nvfp4_amax_fakequant(A, 1, 4, 32, 1, 9, A, A, None, None, None, None), 5),
+    (lambda L: L.nvfp4_amax_fakequant(A, 1, 4, 32, 1, 2, A, A + 16, None, None, None, None), 3),
     # nvfp4_fakequant(x, G, R, C, amax, mode, rule, y, choice, stream)
     (lambda L: L.nvfp4_fakequant(A, 1, 4, 32, A, 1, 2, None, None, None), 1),
     (lambda L: L.nvfp4_fakequant(A, 1, 4, 32, A, 7, 2, A, None, None), 4),

@@ -249,3 +249,45 @@ def test_parity_scale_on_e4m3_boundary(gpu, mode, rule):
         assert sum(used) >= 100 and len(used) - sum(used) >= 20, (sum(used), len(used))
         x = _boundary_tensor(groups, bpg, seed=bpg)
         U.check_case(x, len(groups), bpg, 16, mode, rule)
+
+
+# ---- amax and quantization in one launch (a grid-wide wait between them) ------------------------
+
+# one group (ragged), several groups of whole warp words (one launch), and several groups whose
+# block count is not a multiple of 32 (the two launches)
+ONE_LAUNCH = [("c1", 256, 1024, 1), ("c2", 517, 4080, 1), ("c4", 128, 1024, 4), ("c4", 129, 1008, 3),
+              ("c5", 301, 8176, 1)]
+
+
+@pytest.mark.parametrize("mode,rule", MODES, ids=MODE_IDS)
+@pytest.mark.parametrize("case", ONE_LAUNCH, ids=lambda c: f"{c[0]}-{c[1]}x{c[2]}x{c[3]}")
+def test_parity_amax_in_the_same_launch(gpu, case, mode, rule):
+    name, rows, cols, groups = case
+    x, (g, r, c) = synth.make(name, rows=rows, cols=cols, groups=groups)
+    n, nb = g * r * c, g * r * c // 16
+    want_amax = O.amax(x, g, r, c)
+    want = O.quantize(x, g, r, c, want_amax, mode, rule)
+    wfq = O.fakequant(x, g, r, c, want_amax, mode, rule)
+    xd = U.to_device_bf16(x)
+    amax, tscale = U.Guarded(4 * g), U.Guarded(4 * g)
+    codes, scales, choice = U.Guarded(n // 2), U.Guarded(nb), U.Guarded((nb + 7) // 8)
+    work = torch.zeros(2, dtype=torch.int32, device="cuda")     # [0] workspace, [1] status
+    nv.nvfp4_amax_quantize(xd.data_ptr(), g, r, c, mode, rule, amax.ptr(), codes.ptr(), scales.ptr(), tscale.ptr(),
+                           choice.ptr(), work[0:1].data_ptr(), work[1:2].data_ptr())
+    torch.cuda.synchronize()
+    assert work[1].item() == 0
+    assert all(b.guards_intact() for b in (amax, tscale, codes, scales, choice)), "write outside an output buffer"
+    U.assert_same("amax", amax.numpy(np.float32), want_amax)
+    U.assert_same("tscale", tscale.numpy(np.float32), want["tscale"])
+    for k, buf in (("codes", codes), ("scales", scales), ("choice", choice)):
+        U.assert_same(k, buf.numpy(), want[k])
+    # fake-quant, twice in a row on the library's own workspace word
+    for _ in range(2):
+        amax2, y, choice2 = U.Guarded(4 * g), U.Guarded(2 * n), U.Guarded((nb + 7) // 8)
+        nv.nvfp4_amax_fakequant(xd.data_ptr(), g, r, c, mode, rule, amax2.ptr(), y.ptr(), choice2.ptr(), None,
+                                work[1:2].data_ptr())
+        torch.cuda.synchronize()
+        assert work[1].item() == 0 and y.guards_intact() and choice2.guards_intact()
+        U.assert_same("amax", amax2.numpy(np.float32), want_amax)
+        U.assert_same("fakequant", y.numpy(np.uint16), wfq["fq"])
+        U.assert_same("fakequant choice", choice2.numpy(), wfq["choice"])
