@@ -487,6 +487,27 @@ def per_config_leg(nv, torch, dev, stream, peak, resident=None):
                 if rep_i >= 2:
                     t_aq.append(dt)
         res["amax_plus_quantize_ms"] = round(statistics.median(t_aq), 5)
+
+        # the same two steps in one launch (grid-wide barrier), flushed or in batches as above
+        work = torch.zeros(2, dtype=torch.int32, device=dev)
+
+        def one_launch():
+            cs = torch.cuda.current_stream(dev).cuda_stream
+            m, rl = variants[-1][1], variants[-1][2]
+            if fq:
+                nv.nvfp4_amax_fakequant(xd, g, r, c, m, rl, amax, y, choice, work[0:1], work[1:2], cs)
+            else:
+                nv.nvfp4_amax_quantize(xd, g, r, c, m, rl, amax, codes, scales, tscale, choice, work[0:1], work[1:2],
+                                       cs)
+
+        one_launch()
+        t_one = []
+        for rep_i in range(8):
+            dt = timed(one_launch, fits_l2)
+            if rep_i >= 2:
+                t_one.append(dt)
+        res["amax_quantize_one_launch_ms"] = round(statistics.median(t_one), 5)
+        res["one_launch_status"] = int(work[1].item())
         out[name] = res
         del xd
         if fq:
