@@ -217,7 +217,10 @@ NVFP4_API nvfp4_status nvfp4_quantize_gemm(const uint16_t* x, int64_t rows, int6
  * m >= 0 is any row count, n a multiple of 128 and k of 256 (else NVFP4_ERR_SHAPE); codes and
  * scales 16-byte aligned, y 32-byte aligned; the tensor-map encoder of the driver must be available (else
  * NVFP4_ERR_CUDA). The accumulation is FP32 inside the tensor core, so y agrees
- * with the exact product to within FP32 accumulation error, not bit for bit. */
+ * with the exact product to within FP32 accumulation error, not bit for bit. Shapes whose m
+ * and n are multiples of 256 run on clusters of two CTAs (tcgen05 cta_group::2, one 256 x 256
+ * output tile per pair, bit-identical to the one-CTA kernel); the cluster launch must be
+ * available (else NVFP4_ERR_CUDA). */
 NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const float* x_tscale,
                                   const uint8_t* w_codes, const uint8_t* w_scales, const float* w_tscale,
                                   int64_t m, int64_t n, int64_t k, float* y, uint32_t* status,

@@ -26,6 +26,7 @@
 //                      tcgen05.mma.kind::mxf4nvf4.block_scale.block16 into the FP32
 //                      accumulator in tensor memory, and commits them to the stage's "empty"
 //                      mbarrier, which releases the slot to the producers.
+// m and n multiples of 256 run on pairs of CTAs instead (gemm_fp4_pair_kernel, below).
 // The epilogue (warps 2-9, two per 32-lane quarter of tensor memory and 128 columns each; in
 // the prologue variant warps 2-5, one per quarter) reads the accumulator with tcgen05.ld,
 // releases it to the MMA lane and scales it by alpha_x * alpha_w while it stores. Every mbarrier wait is bounded: on
@@ -247,6 +248,81 @@ __device__ __forceinline__ void sts16(uint32_t addr, uint4 v) {
 
 __device__ __forceinline__ void sts16b(uint32_t addr, uint16_t v) {
     asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
+// ---- pairs of CTAs (a cluster of two, tcgen05 cta_group::2) ----
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of this CTA's shared variable at `addr` in the shared memory of cluster CTA `rank`.
+__device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
+// 2-D tiled TMA load into this CTA's shared memory whose completion is counted on the pair
+// leader's mbarrier (`bar` is a cluster address). Each CTA loads only its own tiles.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                                 uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {   // one warp per CTA
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// tmem_copy_sf in both CTAs of the pair: each copies from its own shared memory at the same
+// offset into its own tensor memory.
+__device__ __forceinline__ void tmem_copy_sf_pair(uint32_t taddr, uint64_t desc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+
+__device__ __forceinline__ void mma_fp4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Arrive on the mbarrier at the same offset in both CTAs of the pair once the tcgen05
+// operations this thread issued so far have completed.
+__device__ __forceinline__ void mma_commit_both(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+        ::"r"(bar), "h"(static_cast<uint16_t>(3))
+        : "memory");
+}
+
+// The same on this CTA's mbarrier only.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
 }
 
 }  // namespace
@@ -599,6 +675,240 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ---- pairs of CTAs on one 256 x 256 tile (tcgen05 cta_group::2) --------------------------------
+
+// A cluster of two CTAs on two SMs owns a 256 x 256 output tile. CTA rank r loads rows 128 r..
+// of the tile's 256 A rows (its accumulator's rows) and rows 128 r.. of its 256 B rows; the
+// leader (rank 0) issues tcgen05.mma.cta_group::2 (M 256, N 256), which takes A from each CTA's
+// own shared memory and B from both, and accumulates into each CTA's tensor memory. Per CTA
+// and K slice the ring holds 38 KiB instead of 54 for the same MMA work: a third less traffic
+// from L2, which the single-CTA kernel draws at about 12 TB/s against a measured read
+// bandwidth of 15-17 TB/s. Each CTA stages the scales of its own A rows and of all 256 B rows
+// (its accumulator needs them all); two lanes of the leader (warps 10 and 11, two MMAs' scales
+// each) move both CTAs' scales into their tensor memory with tcgen05.cp.cta_group::2 as soon
+// as the scale tiles have landed ("sffull", separate from the code tiles' "full"). Used by
+// nvfp4_gemm and nvfp4_gemm_bf16 when m and n are multiples of 256; bit-identical to the
+// single-CTA kernel.
+constexpr int kStagesP = 5;
+constexpr uint32_t kAP = 128 * 128, kBP = 128 * 128, kSfaP = 4 * 512, kSfbP = 8 * 512;
+constexpr uint32_t kStageP = kAP + kBP + kSfaP + kSfbP;             // 38912, a multiple of 1024
+constexpr uint32_t kDynSmemP = kStagesP * kStageP + 1024;
+constexpr uint32_t kColSfaP = 256, kColSfbP = 256 + 16 * kStagesP;  // 256..335, 336..495
+constexpr uint32_t kIdescP = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(256 >> 3) << 17) |
+                             (static_cast<uint32_t>(256 >> 4) << 24);
+constexpr int kWarpsP = 12;   // producer, MMA, eight epilogue warps, two scale-copy warps
+static_assert(kColSfbP + 32 * kStagesP <= kTmemCols, "tensor-memory columns");
+
+// Grid: clusters of 2; cluster c takes 256 x 256 tiles c, c + clusters, ... (tm = t / (n / 256),
+// tn = t % (n / 256)). tmap_a / tmap_b: codes as [rows, k/2] bytes in boxes of 128 bytes x 128
+// rows, 128-byte swizzle; tmap_sa / tmap_sb: the tiled scale buffers viewed as
+// [rows * k / 4096, 256] bytes in boxes of 256 bytes x 8 rows (the four 512-byte scale tiles of
+// a 128-row tile and a 256-element K slice).
+template <bool BF16>
+__global__ void __launch_bounds__(32 * kWarpsP, 1)
+    gemm_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                         const __grid_constant__ CUtensorMap tmap_sa, const __grid_constant__ CUtensorMap tmap_sb,
+                         const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full[kStagesP], empty[kStagesP], sfready[kStagesP], sffull[kStagesP], acc_full,
+        acc_empty, drain;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ volatile uint32_t stop_sh;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_rank();
+    const int64_t n_ct4 = p.k / 256;   // 2 KiB runs of scale tiles per 128 rows
+    const int nk = static_cast<int>(p.k / kBK);
+    const int64_t ntn = p.n / 256, ntiles = (p.m / 256) * ntn;
+    const int64_t cluster_id = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    const uint32_t full0 = smem_u32(&full[0]), empty0 = smem_u32(&empty[0]), sfr0 = smem_u32(&sfready[0]);
+    const uint32_t accf = smem_u32(&acc_full), acce = smem_u32(&acc_empty), drain_bar = smem_u32(&drain);
+    const uint32_t sff0 = smem_u32(&sffull[0]);
+    const uint32_t full0_lead = map_rank(full0, 0), acce_lead = map_rank(acce, 0), sff0_lead = map_rank(sff0, 0);
+
+    if (warp == 1) tmem_alloc_pair(smem_u32(&tmem_base_sh), kTmemCols);
+    if (tid == 0) {
+        for (int s = 0; s < kStagesP; ++s) {
+            mbar_init(full0 + 8 * s, 1);   // the leader's counts both CTAs' bytes
+            mbar_init(empty0 + 8 * s, 1);
+            mbar_init(sfr0 + 8 * s, 2);
+            mbar_init(sff0 + 8 * s, 1);
+        }
+        mbar_init(accf, 1);
+        mbar_init(acce, 16);               // the leader's: eight epilogue warps in each CTA
+        mbar_init(drain_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        stop_sh = 0;
+    }
+    tc_fence_before();
+    cluster_sync_all();   // both CTAs' barriers are initialised and their tensor memory allocated
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    if (warp == 0) {
+        if (lane == 0) {   // producer: this CTA's tiles into its ring, completion on the leader's "full"
+            int g = 0;
+            for (int64_t t = cluster_id; t < ntiles && !stop_sh; t += nclusters) {
+                const int64_t tm = t / ntn, tn = t % ntn;
+                const int64_t rt_a = 2 * tm + rank, rt_b = 2 * tn;   // 128-row tiles
+                for (int ks = 0; ks < nk; ++ks, ++g) {
+                    const int s = g % kStagesP;
+                    const uint32_t u = static_cast<uint32_t>(g / kStagesP);
+                    if (g >= kStagesP && !mbar_wait(empty0 + 8 * s, (u - 1) & 1)) {
+                        stop_sh = 1;
+                        break;
+                    }
+                    const uint32_t fb = full0_lead + 8 * s, sb = sff0_lead + 8 * s;
+                    const uint32_t sA = sbase + s * kStageP, sB = sA + kAP;
+                    const uint32_t sSFA = sB + kBP, sSFB = sSFA + kSfaP;
+                    if (rank == 0) {   // both CTAs' bytes: the scale tiles on "sffull", the codes on "full"
+                        mbar_expect_tx(sff0 + 8 * s, 2 * (kSfaP + kSfbP));
+                        mbar_expect_tx(full0 + 8 * s, 2 * (kAP + kBP));
+                    }
+                    tma_load_2d_pair(sSFA, &tmap_sa, 0, static_cast<int32_t>((rt_a * n_ct4 + ks) * 8), sb);
+                    tma_load_2d_pair(sSFB, &tmap_sb, 0, static_cast<int32_t>((rt_b * n_ct4 + ks) * 8), sb);
+                    tma_load_2d_pair(sSFB + kSfbP / 2, &tmap_sb, 0,
+                                     static_cast<int32_t>(((rt_b + 1) * n_ct4 + ks) * 8), sb);
+                    tma_load_2d_pair(sA, &tmap_a, ks * (kBK / 2), static_cast<int32_t>(rt_a * 128), fb);
+                    tma_load_2d_pair(sB, &tmap_b, ks * (kBK / 2), static_cast<int32_t>((rt_b + rank) * 128), fb);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {   // MMA issuer (leader only), slots unrolled as in the single-CTA kernel
+            const int64_t my_tiles = (ntiles - cluster_id + nclusters - 1) / nclusters;
+            const int64_t total = my_tiles * nk;
+            const uint64_t dA0 = smem_desc_sw128(sbase), dB0 = smem_desc_sw128(sbase + kAP);
+            constexpr uint64_t kSlot = kStageP >> 4;
+            int64_t gg = 0;
+            int ks = 0, tile_j = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            while (gg < total && ok) {
+#pragma unroll
+                for (int s = 0; s < kStagesP; ++s) {
+                    if (gg >= total) break;
+                    if (ks == 0 && tile_j > 0) {   // both CTAs' epilogues have drained tile tile_j - 1
+                        if (!mbar_wait(acce, static_cast<uint32_t>(tile_j - 1) & 1)) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (!mbar_wait(sfr0 + 8 * s, phase) || !mbar_wait(full0 + 8 * s, phase)) {   // scales, codes
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t ca = tmem + kColSfaP + 16 * s, cb = tmem + kColSfbP + 32 * s;
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj)
+                        mma_fp4_pair(tmem, dA0 + s * kSlot + 2 * jj, dB0 + s * kSlot + 2 * jj, kIdescP, ca + 4 * jj,
+                                     cb + 8 * jj, (ks | jj) != 0);
+                    mma_commit_both(empty0 + 8 * s);   // releases the slot in both CTAs
+                    ++gg;
+                    if (++ks == nk) {
+                        ks = 0;
+                        ++tile_j;
+                        mma_commit_both(accf);
+                    }
+                }
+                phase ^= 1;
+            }
+            if (!ok) stop_sh = 1;
+            mma_commit_pair(drain_bar);
+            if (!mbar_wait(drain_bar, 0)) stop_sh = 1;
+        }
+    } else if (warp >= kWarpsP - 2) {
+        if (lane == 0 && rank == 0) {   // scale copies into both CTAs' tensor memory (leader only)
+            const int j0 = (warp - (kWarpsP - 2)) * 2;   // this lane copies the scales of MMAs j0, j0 + 1
+            const int64_t my_tiles = (ntiles - cluster_id + nclusters - 1) / nclusters;
+            const int64_t total = my_tiles * nk;
+            const uint64_t dSA0 = smem_desc(sbase + kAP + kBP, 16, 128);
+            const uint64_t dSB0 = smem_desc(sbase + kAP + kBP + kSfaP, 16, 128);
+            constexpr uint64_t kSlot = kStageP >> 4;
+            int64_t gg = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            while (gg < total && ok) {
+#pragma unroll
+                for (int s = 0; s < kStagesP; ++s) {
+                    if (gg >= total) break;
+                    // the leader's "full" completes once both CTAs' bytes have landed, which is
+                    // after the MMAs that last read this slot's scale columns have finished
+                    if (!mbar_wait(sff0 + 8 * s, phase)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t ca = tmem + kColSfaP + 16 * s, cb = tmem + kColSfbP + 32 * s;
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const int jj = j0 + i;
+                        tmem_copy_sf_pair(ca + 4 * jj, dSA0 + s * kSlot + 32 * jj);
+                        tmem_copy_sf_pair(cb + 8 * jj, dSB0 + s * kSlot + 32 * jj);             // B rows 0..127
+                        tmem_copy_sf_pair(cb + 8 * jj + 4, dSB0 + s * kSlot + 128 + 32 * jj);   // 128..255
+                    }
+                    mma_commit_pair(sfr0 + 8 * s);
+                    ++gg;
+                }
+                phase ^= 1;
+            }
+            if (!ok) stop_sh = 1;
+        }
+    } else {   // epilogue, warps 2-9: lane quarter warp % 4, columns 0..127 (warps 2-5) or 128..255
+        const int q = warp & 3;
+        const int c0 = warp >= 6 ? 128 : 0;
+        int j = 0;
+        for (int64_t t = cluster_id; t < ntiles && !stop_sh; t += nclusters, ++j) {
+            const int64_t tm = t / ntn, tn = t % ntn;
+            uint32_t ok = 1;
+            if (lane == 0) ok = mbar_wait(accf, j & 1);
+            if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+                stop_sh = 1;
+                break;
+            }
+            tc_fence_after();
+            const float alpha = __ldg(p.x_tscale) * __ldg(p.w_tscale);
+            const int64_t off = (tm * 256 + 128 * rank + 32 * q + lane) * p.n + tn * 256 + c0;
+            const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16) + c0;
+            uint32_t r0[64], r1[64];
+            tmem_ld64(trow, r0);
+            tmem_ld64(trow + 64, r1);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acce_lead);   // the accumulator is free before any store
+            if constexpr (BF16) {   // BF16 result and its amax, as in the single-CTA kernel
+                uint32_t mag = 0;
+                uint16_t* yb = p.y16 + off;
+#pragma unroll
+                for (int e = 0; e < 64; e += 16) st_v16bf(yb + e, r0 + e, alpha, mag);
+#pragma unroll
+                for (int e = 0; e < 64; e += 16) st_v16bf(yb + 64 + e, r1 + e, alpha, mag);
+                if (p.y_amax != nullptr) {
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) mag = max(mag, __shfl_xor_sync(0xFFFFFFFFu, mag, o));
+                    if (lane == 0 && mag != 0)
+                        atomicMax(reinterpret_cast<unsigned int*>(p.y_amax),
+                                  __float_as_uint(__bfloat162float(__float2bfloat16_rn(__uint_as_float(mag)))));
+                }
+            } else {
+                float* yr = p.y + off;
+#pragma unroll
+                for (int e = 0; e < 64; e += 8) st_v8f(yr + e, r0 + e, alpha);
+#pragma unroll
+                for (int e = 0; e < 64; e += 8) st_v8f(yr + 64 + e, r1 + e, alpha);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();   // the leader has drained the MMAs that write both CTAs' tensor memory
+    if (stop_sh && tid == 0 && p.status != nullptr) atomicOr(p.status, NVFP4_GEMM_TIMEOUT);
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
+}
+
 // ---- host side -----------------------------------------------------------------------------------
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -646,6 +956,84 @@ nvfp4_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const Gem
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// Tensor map of a tiled scale buffer of `rows` operand rows (a multiple of 128) and k columns
+// (a multiple of 256), viewed as [rows * k / 4096, 256] bytes and read in boxes of 256 bytes x 8
+// rows: the 2 KiB run of four 512-byte scale tiles that a 128-row tile and a 256-element K slice
+// own.
+bool scales_map(CUtensorMap* map, const void* base, int64_t rows, int64_t k) {
+    EncodeTiledFn enc = encode_fn();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[2] = {256u, static_cast<cuuint64_t>(rows / 128 * (k / 32))};
+    const cuuint64_t strides[1] = {256u};
+    const cuuint32_t box[2] = {256u, 8u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Clusters of two CTAs that can be resident at once on the current device (a GPC with an odd
+// number of SMs leaves one unpaired), found once per device.
+int pair_clusters() {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+    if (dev < 64 && cached[dev] > 0) return cached[dev];
+    int sms = 0, active = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(32 * kWarpsP);
+    cfg.dynamicSmemBytes = kDynSmemP;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&active, gemm_fp4_pair_kernel<false>, &cfg) != cudaSuccess || active < 1) {
+        cudaGetLastError();
+        active = sms / 2;
+    }
+    if (dev < 64) cached[dev] = active;
+    return active;
+}
+
+template <bool BF16>
+nvfp4_status launch_gemm_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msa,
+                              const CUtensorMap& msb, const GemmParams& p, cudaStream_t stream) {
+    if (cudaFuncSetAttribute(gemm_fp4_pair_kernel<BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmemP) !=
+        cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    const int active = pair_clusters();
+    if (active < 1) return NVFP4_ERR_CUDA;
+    const int64_t tiles = (p.m / 256) * (p.n / 256);
+    const int64_t clusters = tiles < active ? tiles : active;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters));
+    cfg.blockDim = dim3(32 * kWarpsP);
+    cfg.dynamicSmemBytes = kDynSmemP;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gemm_fp4_pair_kernel<BF16>, ma, mb, msa, msb, p) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+// The pair kernel takes shapes whose 256 x 256 tiles cover the output exactly and whose scale
+// views have row counts that fit the tensor map's 32-bit coordinates.
+bool use_pair(int64_t m, int64_t n, int64_t k) {
+    return m % 256 == 0 && n % 256 == 0 && m / 128 * (k / 32) < (int64_t(1) << 31) &&
+           n / 128 * (k / 32) < (int64_t(1) << 31);
+}
+
 bool aligned16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
 bool aligned4(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 3u) == 0; }
 
@@ -681,8 +1069,12 @@ nvfp4_status gemm_prequantized(const uint8_t* x_codes, const uint8_t* x_scales, 
     // the amax is an atomic maximum over the tiles: it starts from +0 in stream order
     if (y_amax != nullptr && cudaMemsetAsync(y_amax, 0, sizeof(float), stream) != cudaSuccess) return NVFP4_ERR_CUDA;
     if (empty) return NVFP4_OK;
-    CUtensorMap ma, mb;
-    if (!codes_map(&ma, x_codes, m, k / 2, kBM) || !codes_map(&mb, w_codes, n, k / 2, kBN)) return NVFP4_ERR_CUDA;
+    const bool pair = use_pair(m, n, k);
+    CUtensorMap ma, mb, msa, msb;
+    if (!codes_map(&ma, x_codes, m, k / 2, pair ? 128u : static_cast<uint32_t>(kBM)) ||
+        !codes_map(&mb, w_codes, n, k / 2, pair ? 128u : static_cast<uint32_t>(kBN)))
+        return NVFP4_ERR_CUDA;
+    if (pair && (!scales_map(&msa, x_scales, m, k) || !scales_map(&msb, w_scales, n, k))) return NVFP4_ERR_CUDA;
     GemmParams p{};
     p.x_scales = x_scales;
     p.x_tscale = x_tscale;
@@ -695,6 +1087,8 @@ nvfp4_status gemm_prequantized(const uint8_t* x_codes, const uint8_t* x_scales, 
     p.m = m;
     p.n = n;
     p.k = k;
+    if (pair) return y16 != nullptr ? launch_gemm_pair<true>(ma, mb, msa, msb, p, stream)
+                                    : launch_gemm_pair<false>(ma, mb, msa, msb, p, stream);
     if (y16 != nullptr) return launch_gemm<false, true, kMse, true>(ma, mb, p, stream);
     return launch_gemm<false, true, kMse>(ma, mb, p, stream);
 }
