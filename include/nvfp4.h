@@ -169,8 +169,8 @@ NVFP4_API nvfp4_status nvfp4_fakequant(const uint16_t* x, int64_t groups, int64_
  *   status     NULL, or a device word; NVFP4_QUANT_TIMEOUT is or-ed in on a timed-out
  *              grid-wide wait                                                        (in/out)
  * Group layouts the grouped quantizer does not take (several groups whose block count is not
- * a multiple of 32), and empty tensors, run as the two separate launches. Errors as
- * nvfp4_quantize, plus NVFP4_ERR_CUDA when the cooperative launch is refused. */
+ * a multiple of 32), empty tensors, and devices that refuse the cooperative launch (the grid
+ * cannot be resident at once) run as the two separate launches. Errors as nvfp4_quantize. */
 NVFP4_API nvfp4_status nvfp4_amax_quantize(const uint16_t* x, int64_t groups, int64_t rows, int64_t cols,
                                            nvfp4_mode mode, nvfp4_rule rule, float* amax, uint8_t* codes,
                                            uint8_t* scales, float* tscale, uint8_t* choice, uint32_t* workspace,
@@ -219,8 +219,8 @@ NVFP4_API nvfp4_status nvfp4_quantize_gemm(const uint16_t* x, int64_t rows, int6
  * NVFP4_ERR_CUDA). The accumulation is FP32 inside the tensor core, so y agrees
  * with the exact product to within FP32 accumulation error, not bit for bit. Shapes whose m
  * and n are multiples of 256 run on clusters of two CTAs (tcgen05 cta_group::2, one 256 x 256
- * output tile per pair, bit-identical to the one-CTA kernel); the cluster launch must be
- * available (else NVFP4_ERR_CUDA). */
+ * output tile per pair, bit-identical to the one-CTA kernel), or on one CTA per tile when
+ * the device refuses the cluster launch. */
 NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* x_codes, const uint8_t* x_scales, const float* x_tscale,
                                   const uint8_t* w_codes, const uint8_t* w_scales, const float* w_tscale,
                                   int64_t m, int64_t n, int64_t k, float* y, uint32_t* status,

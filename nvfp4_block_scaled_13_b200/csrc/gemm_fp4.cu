@@ -972,6 +972,9 @@ bool scales_map(CUtensorMap* map, const void* base, int64_t rows, int64_t k) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A pair launch that was refused (no cluster of two can be resident, or the launch failed).
+constexpr nvfp4_status kPairRefused = static_cast<nvfp4_status>(1000);
+
 // Clusters of two CTAs that can be resident at once on the current device (a GPC with an odd
 // number of SMs leaves one unpaired), found once per device.
 int pair_clusters() {
@@ -1007,7 +1010,7 @@ nvfp4_status launch_gemm_pair(const CUtensorMap& ma, const CUtensorMap& mb, cons
         cudaSuccess)
         return NVFP4_ERR_CUDA;
     const int active = pair_clusters();
-    if (active < 1) return NVFP4_ERR_CUDA;
+    if (active < 1) return kPairRefused;
     const int64_t tiles = (p.m / 256) * (p.n / 256);
     const int64_t clusters = tiles < active ? tiles : active;
     cudaLaunchConfig_t cfg = {};
@@ -1022,8 +1025,10 @@ nvfp4_status launch_gemm_pair(const CUtensorMap& ma, const CUtensorMap& mb, cons
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gemm_fp4_pair_kernel<BF16>, ma, mb, msa, msb, p) != cudaSuccess)
-        return NVFP4_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, gemm_fp4_pair_kernel<BF16>, ma, mb, msa, msb, p) != cudaSuccess) {
+        cudaGetLastError();   // cluster launch refused: the caller runs the one-CTA kernel
+        return kPairRefused;
+    }
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
@@ -1087,8 +1092,13 @@ nvfp4_status gemm_prequantized(const uint8_t* x_codes, const uint8_t* x_scales, 
     p.m = m;
     p.n = n;
     p.k = k;
-    if (pair) return y16 != nullptr ? launch_gemm_pair<true>(ma, mb, msa, msb, p, stream)
-                                    : launch_gemm_pair<false>(ma, mb, msa, msb, p, stream);
+    if (pair) {
+        const nvfp4_status ps = y16 != nullptr ? launch_gemm_pair<true>(ma, mb, msa, msb, p, stream)
+                                               : launch_gemm_pair<false>(ma, mb, msa, msb, p, stream);
+        if (ps != kPairRefused) return ps;
+        // the one-CTA kernel reads B in boxes of 256 rows
+        if (!codes_map(&ma, x_codes, m, k / 2, kBM) || !codes_map(&mb, w_codes, n, k / 2, kBN)) return NVFP4_ERR_CUDA;
+    }
     if (y16 != nullptr) return launch_gemm<false, true, kMse, true>(ma, mb, p, stream);
     return launch_gemm<false, true, kMse>(ma, mb, p, stream);
 }

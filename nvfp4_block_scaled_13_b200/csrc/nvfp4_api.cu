@@ -141,6 +141,9 @@ nvfp4_status dispatch_quant(nvfp4_mode mode, nvfp4_rule rule, const nvfp4::Quant
     }
 }
 
+// Internal: a cooperative or cluster launch was refused, and the caller takes its other path.
+constexpr nvfp4_status NVFP4_ERR_UNSUPPORTED_LAUNCH = static_cast<nvfp4_status>(1000);
+
 // Barrier counter of nvfp4_amax_quantize / nvfp4_amax_fakequant calls without a workspace:
 // library memory (one per device), so those calls allocate nothing; they must not overlap.
 __device__ __align__(256) uint32_t g_amax_quant_scratch[64];
@@ -154,8 +157,10 @@ nvfp4_status launch_quant_amax(const nvfp4::QuantParams& p, uint32_t* arrive, ui
     nvfp4::QuantParams pp = p;
     void* args[] = {&pp, &arrive, &status};
     if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), grid, dim3(kThreads), args, 0, stream) !=
-        cudaSuccess)
-        return NVFP4_ERR_CUDA;
+        cudaSuccess) {
+        cudaGetLastError();   // refused (e.g. the grid cannot be resident): the caller runs two launches
+        return NVFP4_ERR_UNSUPPORTED_LAUNCH;
+    }
     return launch_status();
 }
 
@@ -242,8 +247,13 @@ nvfp4_status amax_quant_impl(const uint16_t* x, int64_t groups, int64_t rows, in
     p.choice_bytes = (p.nblocks + 7) / 8;
     p.groups = groups;
     p.gdiv = make_gdiv(groups, bpg, p.nblocks);
-    return fq ? dispatch_quant_amax<true>(mode, rule, p, workspace, status, stream)
-              : dispatch_quant_amax<false>(mode, rule, p, workspace, status, stream);
+    st = fq ? dispatch_quant_amax<true>(mode, rule, p, workspace, status, stream)
+            : dispatch_quant_amax<false>(mode, rule, p, workspace, status, stream);
+    if (st != NVFP4_ERR_UNSUPPORTED_LAUNCH) return st;
+    st = nvfp4_amax(x, groups, rows, cols, amax, stream);   // the two launches
+    if (st != NVFP4_OK) return st;
+    return fq ? nvfp4_fakequant(x, groups, rows, cols, amax, mode, rule, y, choice, stream)
+              : nvfp4_quantize(x, groups, rows, cols, amax, mode, rule, codes, scales, tscale, choice, stream);
 }
 
 }  // namespace
