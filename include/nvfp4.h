@@ -201,8 +201,8 @@ NVFP4_API nvfp4_status nvfp4_quantize_gemm(const uint16_t* x, int64_t rows, int6
                                            float* tscale, uint8_t* choice, cudaStream_t stream);
 
 /* Bit set in a GEMM's status word when one of the kernel's bounded waits for the tensor core
- * timed out (about two seconds); the kernel then stops, frees its tensor memory and leaves y
- * partly written. */
+ * timed out (about two seconds); the kernel then stops, lets the copies it already issued land
+ * (again bounded), frees its tensor memory and leaves y partly written. */
 #define NVFP4_GEMM_TIMEOUT 1u
 
 /* Block-scaled FP4 GEMM on the 5th-generation tensor cores (tcgen05, kind::mxf4nvf4 with

@@ -250,6 +250,18 @@ __device__ __forceinline__ void sts16b(uint32_t addr, uint16_t v) {
     asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
 
+// After a timed-out wait: let the copies this producer issued land before the CTA exits. Slot
+// s last received slice s + kStages * j (j = (issued - 1 - s) / stages); its barriers complete
+// the phase of parity j & 1 once those bytes have arrived. Each wait is bounded.
+__device__ __forceinline__ void drain_copies(uint32_t full0, uint32_t sff0, bool scales_apart, int issued,
+                                             int stages) {
+    for (int s = 0; s < stages && s < issued; ++s) {
+        const uint32_t parity = static_cast<uint32_t>((issued - 1 - s) / stages) & 1u;
+        mbar_wait(full0 + 8 * s, parity);
+        if (scales_apart) mbar_wait(sff0 + 8 * s, parity);
+    }
+}
+
 // ---- pairs of CTAs (a cluster of two, tcgen05 cta_group::2) ----
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -451,6 +463,7 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
                     tma_load_2d(sB, &tmap_b, ks * (kBK / 2), static_cast<int32_t>(tn * kBN), fb);
                 }
             }
+            if (stop_sh) drain_copies(full0, sff0, !QUANT, g, kStages);
         }
     } else if (warp == 1) {
         if (lane == 0) {   // MMA issuer: one thread issues every tcgen05 instruction, so its per-slice
@@ -773,6 +786,9 @@ __global__ void __launch_bounds__(32 * kWarpsP, 1)
                     tma_load_2d_pair(sB, &tmap_b, ks * (kBK / 2), static_cast<int32_t>((rt_b + rank) * 128), fb);
                 }
             }
+            // the leader's barriers count both CTAs' bytes; the closing cluster barrier keeps the
+            // other CTA (and its shared memory) alive until then
+            if (stop_sh && rank == 0) drain_copies(full0, sff0, true, g, kStagesP);
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {   // MMA issuer (leader only), slots unrolled as in the single-CTA kernel
