@@ -123,3 +123,52 @@ def check_case(x: np.ndarray, g: int, r: int, c: int, mode: int, rule: int, amax
         gy = gpu_dequantize(got["codes"], got["scales"], got["tscale"], g, r, c)
         assert_same("dequantize", gy, O.dequantize(want["codes"], want["scales"], want["tscale"], g, r, c))
     return got
+
+
+def host_threads() -> int:
+    try:
+        import os
+
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return 1
+
+
+def oracle_whole(x: np.ndarray, g: int, r: int, c: int, amax_np, mode: int, rule: int, fakequant: bool = False,
+                 threads: int | None = None):
+    """The oracle's quantization (fakequant=False: codes, scales, tscale, choice; True: fq,
+    choice) of the whole [g, r, c] tensor, computed as independent row ranges on host threads.
+
+    Blocks depend only on their group's amax, so a row range quantized alone gives the same
+    bytes as the whole tensor (a CPU test pins this); the C oracle releases the interpreter
+    lock while it runs, so the ranges run in parallel."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    threads = threads or host_threads()
+    n, nb, bpr = g * r * c, g * r * c // 16, c // 16
+    parts = max(1, -(-threads // g))
+    tasks = [(gi, r * k // parts, r * (k + 1) // parts) for gi in range(g) for k in range(parts)]
+    tasks = [t for t in tasks if t[2] > t[1]]
+    amax_np = np.ascontiguousarray(amax_np, np.float32)
+
+    def run(t):
+        gi, lo, hi = t
+        xs = x[(gi * r + lo) * c:(gi * r + hi) * c]
+        fn = O.fakequant if fakequant else O.quantize
+        return t, fn(xs, 1, hi - lo, c, amax_np[gi:gi + 1], mode, rule)
+
+    out = dict(fq=np.empty(n, np.uint16)) if fakequant else dict(
+        codes=np.empty(n // 2, np.uint8), scales=np.empty(nb, np.uint8), tscale=np.zeros(g, np.float32))
+    bits = np.empty(nb, np.uint8)
+    with ThreadPoolExecutor(min(threads, len(tasks))) as ex:
+        for (gi, lo, hi), o in ex.map(run, tasks):
+            e0, e1 = (gi * r + lo) * c, (gi * r + hi) * c
+            if fakequant:
+                out["fq"][e0:e1] = o["fq"]
+            else:
+                out["codes"][e0 // 2:e1 // 2] = o["codes"]
+                out["scales"][e0 // 16:e1 // 16] = o["scales"]
+                out["tscale"][gi] = o["tscale"][0]
+            bits[e0 // 16:e1 // 16] = np.unpackbits(o["choice"], bitorder="little")[:(hi - lo) * bpr]
+    out["choice"] = np.packbits(bits, bitorder="little")
+    return out
