@@ -33,6 +33,8 @@ MUTANTS = {
     "decode_scale_transposed": ("c->d = nvo_e4m3_to_f32(c->s) * alpha;", "c->d = nvo_e4m3_to_f32(c->s) / alpha;"),
     "error_against_scaled_values": ("c->e[i] = fmaf(-v, c->d, x[i]);", "c->e[i] = y - v;"),
     "error_drops_scale": ("c->e[i] = fmaf(-v, c->d, x[i]);", "c->e[i] = x[i] - v;"),
+    # the other reading of the error term: the dequantized value rounded before the subtraction
+    "error_rounds_product_first": ("c->e[i] = fmaf(-v, c->d, x[i]);", "c->e[i] = x[i] - c->q[i];"),
     "zero_sign_dropped": ("uint8_t sign = signbit(y) ? 0x8u : 0x0u;", "uint8_t sign = (y < 0) ? 0x8u : 0x0u;"),
     "kl_reversed": ("acc += p * (logp - logq);", "acc += q * (logq - logp);"),
     "kl_grad_sign": ("grad[r * vocab + v] = grad_scale * (q - p);", "grad[r * vocab + v] = grad_scale * (p - q);"),

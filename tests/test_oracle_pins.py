@@ -509,3 +509,97 @@ def test_row_ranges_quantize_like_the_whole_tensor():
     for k in ("codes", "scales", "choice"):
         assert np.array_equal(np.concatenate([q[k] for q in got]), whole[k]), k
     assert all(np.array_equal(q["tscale"], whole["tscale"]) for q in got)
+
+
+# ---- the error term: the exact difference rounded once --------------------------------------
+
+def _exact_block_choice(xs, alpha, rule, once):
+    """Both candidates of one Four Over Six block in exact rational arithmetic, each binary32
+    operation of the pipeline rounded to nearest even as the reading states (tests/exact.py),
+    with the error term either the exact difference x - v d rounded once (once=True) or the
+    dequantized value rounded first, RN(x - RN(v d)). Returns (choose 4, err_4, err_6)."""
+    R = X.round_f32
+    m = max(abs(v) for v in xs)
+    errs = {}
+    for K in (6, 4):
+        beta = R(K * alpha)
+        t = R(m / beta) if beta > 0 else F(0)
+        s = X.E4M3[X.nearest_ties_even(t, X.E4M3)[0]]
+        d = R(s * alpha)
+        r = min(R(1 / d), X.FLT_MAX) if d > 0 else F(0)
+        acc = [F(0), F(0)]
+        emax = F(0)
+        for i, xv in enumerate(xs):
+            y = R(xv * r)
+            v = X.E2M1_GRID[X.nearest_ties_even(abs(y), X.E2M1_GRID)[0]] * (-1 if y < 0 else 1)
+            e = R(xv - v * d) if once else R(xv - R(v * d))
+            if rule == 0:
+                emax = max(emax, abs(e))
+            elif rule == 1:
+                acc[i & 1] = R(acc[i & 1] + abs(e))
+            else:
+                acc[i & 1] = R(e * e + acc[i & 1])
+        errs[K] = emax if rule == 0 else R(acc[0] + acc[1])
+    return errs[4] < errs[6], errs[4], errs[6]
+
+
+def _error_reading_blocks():
+    path = os.path.join(GOLDEN, "error_reading_blocks.txt")
+    out = []
+    for ln in open(path):
+        if ln.startswith("#") or not ln.strip():
+            continue
+        f = ln.split()
+        alpha = np.array([int(f[1], 16)], np.uint32).view(np.float32)
+        x = np.array([int(v, 16) for v in f[2:18]], np.uint16)
+        out.append((int(f[0]), alpha, x))
+    return out
+
+
+def test_error_term_is_the_exact_difference_rounded_once():
+    """Four Over Six, Method > Adaptive block scaling algorithm: each candidate's error is
+    measured against the original high-precision values. The page does not fix the rounding:
+    this build reads it as e_i = RN(x_i - v_i d), the exact difference between the original
+    value and the dequantized value, rounded once; the other plausible reading rounds the
+    dequantized value first, RN(x_i - RN(v_i d)). The reading, not the page, decides. The
+    fixture holds blocks (inputs only) on which the two readings choose different candidates;
+    the choice of each reading is recomputed here in exact rational arithmetic, and the oracle
+    must make the first reading's choice on every block, so a two-rounding oracle fails."""
+    blocks = _error_reading_blocks()
+    assert len(blocks) >= 30
+    rules_seen = set()
+    for rule, alpha_f, x in blocks:
+        xs = [X.f32_value(float(v)) for v in ((x.astype(np.uint32) << 16).view(np.float32))]
+        alpha = X.f32_value(float(alpha_f[0]))
+        once, e4, e6 = _exact_block_choice(xs, alpha, rule, True)
+        twice, _, _ = _exact_block_choice(xs, alpha, rule, False)
+        assert once != twice, "fixture block does not separate the readings"
+        # the oracle, given the block as a one-group tensor whose amax gives this alpha
+        c4 = O.block_candidate([float(v) for v in xs], float(alpha_f[0]), 4.0, rule)
+        c6 = O.block_candidate([float(v) for v in xs], float(alpha_f[0]), 6.0, rule)
+        assert X.f32_value(c4.err) == e4 and X.f32_value(c6.err) == e6, (rule, float(c4.err), float(e4))
+        assert (c4.err < c6.err) == once
+        rules_seen.add(rule)
+    assert rules_seen == {0, 1, 2}
+
+
+def test_error_term_per_element_in_exact_rationals():
+    """Per element of random blocks: the oracle's e_i equals the exact x_i - v_i d rounded once
+    to binary32, and (so that the check can tell the readings apart) a good share of those
+    elements differ from RN(x_i - RN(v_i d))."""
+    rng = np.random.default_rng(23)
+    differ = checked = 0
+    for _ in range(60):
+        x = bf16_bits(list(rng.standard_normal(16) * rng.lognormal(0, 1)))
+        xs = [X.f32_value(float(v)) for v in ((x.astype(np.uint32) << 16).view(np.float32))]
+        alpha = float(f32(max(abs(float(v)) for v in xs) * rng.uniform(1, 3) / 1536.0))
+        for K in (6.0, 4.0):
+            c = O.block_candidate([float(v) for v in xs], alpha, K, 2)
+            d = X.f32_value(c.d)
+            for i in range(16):
+                v = X.E2M1_GRID[c.code[i] & 7] * (-1 if c.code[i] & 8 else 1)
+                want = X.round_f32(xs[i] - v * d)
+                assert X.f32_value(c.e[i]) == want, (i, c.e[i], float(want))
+                differ += X.round_f32(xs[i] - X.round_f32(v * d)) != want
+                checked += 1
+    assert differ >= checked // 20, (differ, checked)
