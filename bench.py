@@ -8,7 +8,9 @@ One step is one pass of the whole hot path over one tensor resident in HBM:
     choice bits) -> nvfp4_dequantize,
 on the 1 GiB workload: BF16 65536 x 8192, N(0,1), 1% zero blocks, 1% blocks x1e-6.
 Each rank quantizes its own tensor (weak scaling, no collective on the data path).
-`value` is input GB/s over all ranks: ranks * 2 * numel / (max over ranks of step time).
+`value` is the metric's quantize-kernel input GB/s with the amax given: ranks * 2 * numel /
+(max over ranks of the quantize launch's mean CUDA-event time inside the timed steps);
+`step_input_GBps` is the same over the whole step (amax + quantize + dequantize).
 
 Rank 0 prints one JSON line with the roofline of the dominant kernel (quantize), measured
 live with CUDA events; the end-to-end number through the public API with host buffers;
@@ -221,17 +223,21 @@ def host_threads() -> int:
         return max(1, os.cpu_count() or 1)
 
 
-def oracle_step(x_rows: np.ndarray, rows: int, cols: int, threads: int = 1):
-    """amax, quantize (amax given) and dequantize by the oracle, its C functions called on
-    `threads` row ranges at once (the oracle's calls release the interpreter lock and blocks
-    are independent, so the ranges give the same bytes as one call over all rows)."""
+def oracle_step(x_rows: np.ndarray, rows: int, cols: int, threads: int = 1, amax=None):
+    """The oracle's quantize (Four Over Six, MSE) of `rows` rows with the tensor amax given,
+    the metric's operation; with amax=None, amax + quantize + dequantize (the whole path). Its
+    C functions are called on `threads` row ranges at once (the oracle's calls release the
+    interpreter lock and blocks are independent, so the ranges give the same bytes as one call
+    over all rows)."""
     import oracle as O
 
     O.lib()
+    whole = amax is None
     if threads <= 1:
-        a = O.amax(x_rows, 1, rows, cols)
+        a = O.amax(x_rows, 1, rows, cols) if whole else amax
         q = O.quantize(x_rows, 1, rows, cols, a, MODE, RULE)
-        O.dequantize(q["codes"], q["scales"], q["tscale"], 1, rows, cols)
+        if whole:
+            O.dequantize(q["codes"], q["scales"], q["tscale"], 1, rows, cols)
         return
     from concurrent.futures import ThreadPoolExecutor
 
@@ -239,29 +245,37 @@ def oracle_step(x_rows: np.ndarray, rows: int, cols: int, threads: int = 1):
     bounds = [(lo, hi) for lo, hi in bounds if hi > lo]
     part = lambda lo, hi: x_rows[lo * cols:hi * cols]
     with ThreadPoolExecutor(len(bounds)) as ex:
-        a = np.max(list(ex.map(lambda b: O.amax(part(*b), 1, b[1] - b[0], cols), bounds)), axis=0)
+        a = np.max(list(ex.map(lambda b: O.amax(part(*b), 1, b[1] - b[0], cols), bounds)), axis=0) if whole else amax
 
         def rest(b):
             q = O.quantize(part(*b), 1, b[1] - b[0], cols, a, MODE, RULE)
-            O.dequantize(q["codes"], q["scales"], q["tscale"], 1, b[1] - b[0], cols)
+            if whole:
+                O.dequantize(q["codes"], q["scales"], q["tscale"], 1, b[1] - b[0], cols)
 
         list(ex.map(rest, bounds))
 
 
-def cpu_baseline(x: np.ndarray, cols: int, rows: int = 12288):
-    """The oracle as it stands (C) on the first `rows` rows of the workload: on all host
-    cores (the reported value), and on one thread."""
+def tensor_amax(x: np.ndarray) -> np.ndarray:
+    """max |x| of a BF16 tensor (uint16 bits) as binary32: BF16 magnitudes order like their bits."""
+    m = int(np.max(x & np.uint16(0x7FFF))) if x.size else 0
+    return np.array([m << 16], np.uint32).view(np.float32)
+
+
+def cpu_baseline(x: np.ndarray, cols: int, amax: np.ndarray, rows: int = 12288):
+    """The oracle as it stands (C) on the first `rows` rows of the workload, quantizing with
+    the whole tensor's amax given (the metric's operation): on all host cores (the reported
+    value), and on one thread."""
     xs = np.ascontiguousarray(x[: rows * cols])
     threads = host_threads()
     t0 = time.perf_counter()
-    oracle_step(xs, rows, cols, threads)
+    oracle_step(xs, rows, cols, threads, amax=amax)
     dt_all = time.perf_counter() - t0
     t0 = time.perf_counter()
-    oracle_step(xs, rows, cols, 1)
+    oracle_step(xs, rows, cols, 1, amax=amax)
     dt_one = time.perf_counter() - t0
     return {"value": round(2 * rows * cols / dt_all / GB, 5), "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": f"rows 0..{rows - 1} of the 65536x8192 tensor ({rows * cols / 1e6:.1f} M elements): "
-                      f"amax + 4/6-MSE quantize + dequantize on {threads} threads ({dt_all:.2f} s); "
+                      f"4/6-MSE quantize with the tensor amax given, on {threads} threads ({dt_all:.2f} s); "
                       f"one thread: {dt_one:.1f} s",
             "single_thread": {"value": round(2 * rows * cols / dt_one / GB, 5), "unit": "GB/s"}}
 
@@ -272,30 +286,32 @@ def run_reference(args, rank, world):
         return
     x, (g, r, c) = make_input(0, args.rows)
     threads = host_threads()
+    amax = tensor_amax(x)          # the metric quantizes with the amax given
     # calibrate, then size each step's sample so that the whole run takes about two minutes
     cal_rows = 16 * threads
     t0 = time.perf_counter()
-    oracle_step(np.ascontiguousarray(x[: cal_rows * c]), cal_rows, c, threads)
+    oracle_step(np.ascontiguousarray(x[: cal_rows * c]), cal_rows, c, threads, amax=amax)
     per_row = (time.perf_counter() - t0) / cal_rows
     rows = int(max(threads, min(8192, r // 2, 120.0 / max(1, args.steps + args.warmup) / per_row)))
     for i in range(args.warmup):
         s = (i * rows) % (r - rows)
-        oracle_step(np.ascontiguousarray(x[s * c:(s + rows) * c]), rows, c, threads)
+        oracle_step(np.ascontiguousarray(x[s * c:(s + rows) * c]), rows, c, threads, amax=amax)
     t0 = time.perf_counter()
     for i in range(args.steps):
         s = ((args.warmup + i) * rows) % (r - rows)
-        oracle_step(np.ascontiguousarray(x[s * c:(s + rows) * c]), rows, c, threads)
+        oracle_step(np.ascontiguousarray(x[s * c:(s + rows) * c]), rows, c, threads, amax=amax)
     dt = time.perf_counter() - t0
     value = 2 * rows * c * args.steps / dt / GB
-    sample = (f"{rows} rows x 8192 per step ({rows * c / 1e6:.2f} M elements): amax + 4/6-MSE quantize + "
-              f"dequantize on {threads} threads")
+    sample = (f"{rows} rows x 8192 per step ({rows * c / 1e6:.2f} M elements): 4/6-MSE quantize with the tensor "
+              f"amax given, on {threads} threads")
     print(json.dumps({
         "impl": "reference", "metric": "NVFP4 quantize input GB/s & % of B200 HBM peak; 4/6 overhead vs scale-6",
         "value": round(value, 6), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": f"c5: BF16 {r}x{c} N(0,1), 1% zero blocks, 1% blocks x1e-6; "
-                               "Four Over Six, MSE rule", "shape": [1, r, c], "step": "amax + quantize + dequantize"},
+                               "Four Over Six, MSE rule", "shape": [1, r, c],
+                   "step": "quantize (codes, scales, tscale, choice) of a row sample with the tensor amax given"},
         "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -571,7 +587,11 @@ def run_ours(args, rank, world, local):
     t_quant = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     t_deq = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     step_ms = max_over_ranks(elapsed_ms / args.steps, world)
-    value = world * 2 * n / (step_ms * 1e-3) / GB
+    # the metric: quantize-kernel input GB/s with the amax given, 2N / t_q over all ranks, t_q the
+    # mean CUDA-event time of the quantize launch inside the K timed steps (max over ranks)
+    tq_ms = max_over_ranks(t_quant, world)
+    value = world * 2 * n / (tq_ms * 1e-3) / GB
+    step_value = world * 2 * n / (step_ms * 1e-3) / GB
     launches = 3 * args.steps
 
     # ---- Four Over Six overhead vs scale-6 on the same GPU (quantize kernel, amax given) ----
@@ -658,7 +678,7 @@ def run_ours(args, rank, world, local):
     # ---- CPU oracle on a bounded sample (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(x_np, c, rows=min(12288, r))
+        cpu = cpu_baseline(x_np, c, tensor_amax(x_np), rows=min(12288, r))
 
     if rank == 0:
         peak, peak_kind = measured_peak()
@@ -670,6 +690,11 @@ def run_ours(args, rank, world, local):
             "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(step_ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
+            "value_definition": "quantize-kernel input GB/s with the amax given: ranks * 2N / t_q, t_q the mean "
+                                "CUDA-event time of the nvfp4_quantize launch inside the K timed steps (max over "
+                                "ranks)",
+            "quantize_ms": round(tq_ms, 5),
+            "step_input_GBps": round(step_value, 2),
             "config": {
                 "workload": f"c5: BF16 {r}x{c} ({2 * n / 2**30:.3g} GiB) N(0,1), 1% zero blocks, 1% blocks x1e-6; "
                             "Four Over Six, MSE rule; one tensor per rank",
@@ -708,7 +733,174 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+# ---- profiling tools: one small, self-terminating run of one kernel family -------------------
+# python bench.py --tool case --workload c5 --rows 16384 --mode four_over_six --rule mse --reps 3
+#     amax, quantize (or fakequant / tiled-scale quantize) and dequantize on one workload slice
+# python bench.py --tool gemm --m 8192 --n 4096 --k 4096 --reps 20
+#     the block-scaled FP4 GEMM (pre-quantized, BF16 result, activation quantize, prologue)
+# python bench.py --tool kl --rows 4096 --vocab 131072 --reps 20 [--no-grad]
+#     the QAD distillation loss kernel
+# They print CUDA-event times; ncu captures in profiles/ name these commands.
+
+def tool_case(argv):
+    import torch
+
+    import nvfp4_block_scaled_13_b200 as nv
+    from nvfp4_block_scaled_13_b200 import synth
+
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="c5", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--rows", type=int, default=None)
+    ap.add_argument("--groups", type=int, default=None)
+    ap.add_argument("--mode", default="four_over_six")
+    ap.add_argument("--rule", default="mse")
+    ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--fakequant", action="store_true")
+    ap.add_argument("--gemm-layout", action="store_true", help="nvfp4_quantize_gemm (tiled scales; one group)")
+    a = ap.parse_args(argv)
+
+    nv.load()
+    x, (g, r, c) = synth.make(a.workload, rows=a.rows, groups=a.groups)
+    n, nb = g * r * c, g * r * c // 16
+    xd = torch.from_numpy(x.view(np.int16)).cuda()
+    amax = torch.empty(g, dtype=torch.float32, device="cuda")
+    codes = torch.empty(n // 2, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(nv.gemm_scale_bytes(g * r, c) if a.gemm_layout else nb, dtype=torch.uint8, device="cuda")
+    tscale = torch.empty(g, dtype=torch.float32, device="cuda")
+    choice = torch.empty((nb + 7) // 8, dtype=torch.uint8, device="cuda")
+    y = torch.empty(n, dtype=torch.int16, device="cuda")
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for _ in range(a.reps):
+        ev[0].record()
+        nv.nvfp4_amax(xd, g, r, c, amax)
+        ev[1].record()
+        if a.fakequant:
+            nv.nvfp4_fakequant(xd, g, r, c, amax, a.mode, a.rule, y, choice)
+        elif a.gemm_layout:
+            nv.nvfp4_quantize_gemm(xd, g * r, c, amax, a.mode, a.rule, codes, scales, tscale, choice)
+        else:
+            nv.nvfp4_quantize(xd, g, r, c, amax, a.mode, a.rule, codes, scales, tscale, choice)
+        ev[2].record()
+        if not a.gemm_layout:
+            nv.nvfp4_dequantize(codes, scales, tscale, g, r, c, y)
+        ev[3].record()
+    torch.cuda.synchronize()
+    print(f"{a.workload} [{g},{r},{c}] {a.mode}/{a.rule}: amax {ev[0].elapsed_time(ev[1]):.4f} ms, "
+          f"{'fakequant' if a.fakequant else ('quantize_gemm' if a.gemm_layout else 'quantize')} "
+          f"{ev[1].elapsed_time(ev[2]):.4f} ms, "
+          f"dequantize {ev[2].elapsed_time(ev[3]):.4f} ms (last rep)")
+
+
+
+def tool_gemm(argv):
+    import torch
+
+    import nvfp4_block_scaled_13_b200 as nv
+
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--m", type=int, default=8192)
+    ap.add_argument("--n", type=int, default=4096)
+    ap.add_argument("--k", type=int, default=4096)
+    ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--mode", default="four_over_six")
+    ap.add_argument("--rule", default="mse")
+    a = ap.parse_args(argv)
+
+    nv.load()
+    gen = torch.Generator(device="cuda").manual_seed(7)
+    t = torch.randn(a.m, a.k, device="cuda", generator=gen)
+    t = t / torch.sqrt(torch.rand(a.m, a.k, device="cuda", generator=gen).clamp_min(1e-3))   # heavy tails
+    chan = torch.exp(torch.randn(a.k, device="cuda", generator=gen))
+    x = (t * chan).to(torch.bfloat16).contiguous()
+    w = (torch.randn(a.n, a.k, device="cuda", generator=gen) * 0.02).to(torch.bfloat16).contiguous()
+    del t
+    wq = nv.quantize_for_gemm(w, "four_over_six", "mse")
+    ax = nv.amax(x, 1)
+    xq = nv.quantize_for_gemm(x, a.mode, a.rule, amax_values=ax)
+    y = torch.empty(a.m, a.n, dtype=torch.float32, device="cuda")
+    y16 = torch.empty(a.m, a.n, dtype=torch.bfloat16, device="cuda")
+    y_amax = torch.empty(1, dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+
+    def run_gemm():
+        nv.nvfp4_gemm(xq[0], xq[1], xq[2], wq[0], wq[1], wq[2], a.m, a.n, a.k, y, status, s)
+
+    def run_gemm_bf16():
+        nv.nvfp4_gemm_bf16(xq[0], xq[1], xq[2], wq[0], wq[1], wq[2], a.m, a.n, a.k, y16, y_amax, status, s)
+
+    def run_quant():
+        nv.nvfp4_quantize_gemm(x, a.m, a.k, ax, a.mode, a.rule, xq[0], xq[1], xq[2], None, s)
+
+    def run_prologue():
+        nv.nvfp4_gemm_quantize_x(x, ax, a.mode, a.rule, wq[0], wq[1], wq[2], a.m, a.n, a.k, y, status, s)
+
+    flops = 2.0 * a.m * a.n * a.k
+    out = {"m": a.m, "n": a.n, "k": a.k, "mode": a.mode, "rule": a.rule}
+    for name, fn in (("gemm", run_gemm), ("gemm_bf16", run_gemm_bf16), ("quantize_x", run_quant),
+                     ("prologue", run_prologue)):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(a.reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / a.reps
+        out[name + "_ms"] = round(ms, 4)
+        if name != "quantize_x":
+            out[name + "_tflops"] = round(flops / ms / 1e9, 1)
+    out["status"] = int(status.item())
+    print(json.dumps(out))
+
+
+
+def tool_kl(argv):
+    import torch
+
+    import nvfp4_block_scaled_13_b200 as nv
+
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--rows", type=int, default=4096)
+    ap.add_argument("--vocab", type=int, default=131072)
+    ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--tau", type=float, default=1.0)
+    ap.add_argument("--no-grad", action="store_true")
+    a = ap.parse_args(argv)
+
+    nv.load()
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    t = (torch.randn(a.rows, a.vocab, device="cuda", generator=gen) * 3.0).to(torch.bfloat16)
+    s = (t.float() + torch.randn(a.rows, a.vocab, device="cuda", generator=gen) * 0.3).to(torch.bfloat16)
+    kl = torch.empty(a.rows, dtype=torch.float32, device="cuda")
+    g = None if a.no_grad else torch.empty_like(s)
+    gs = 1.0 / (a.tau * a.rows)
+    for _ in range(3):
+        nv.nvfp4_qad_kl(t, s, a.rows, a.vocab, a.tau, gs, kl, g)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.reps):
+        nv.nvfp4_qad_kl(t, s, a.rows, a.vocab, a.tau, gs, kl, g)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / a.reps
+    n = a.rows * a.vocab
+    algo = 4 * n + (0 if a.no_grad else 2 * n)
+    moved = 4 * n + (0 if a.no_grad else 6 * n)
+    print(json.dumps({"rows": a.rows, "vocab": a.vocab, "grad": not a.no_grad, "ms": round(ms, 4),
+                      "algorithmic_GBps": round(algo / ms / 1e6, 1), "moved_GBps": round(moved / ms / 1e6, 1),
+                      "mean_kl": float(kl.mean())}))
+
+
+
+TOOLS = {"case": tool_case, "gemm": tool_gemm, "kl": tool_kl}
+
+
 def main():
+    if len(sys.argv) > 2 and sys.argv[1] == "--tool":
+        TOOLS[sys.argv[2]](sys.argv[3:])
+        return
     args = parse()
     rank, world, local = dist_setup(args.gpus)
     try:
