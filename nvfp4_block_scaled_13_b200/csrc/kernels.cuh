@@ -230,11 +230,12 @@ __device__ __forceinline__ void cta_max_to(uint32_t* red, uint32_t v, float* out
 // before the launch), then all CTAs meet at a grid-wide barrier on *arrive (zero-filled
 // before the launch), then they quantize as quantize_grouped_kernel does, re-reading their
 // tiles (from L2 when the tensor fits there). The grid must be co-resident (a cooperative
-// launch). The barrier's wait is bounded (about two seconds): on timeout the kernel or-s
-// NVFP4_QUANT_TIMEOUT into *status (nullable) and quantizes nothing.
+// launch). The barrier waits for `expected` arrivals (the library passes gridDim.x). Its wait
+// is bounded (about two seconds): on timeout the CTA or-s NVFP4_QUANT_TIMEOUT into *status
+// (nullable) and quantizes nothing.
 template <bool FOUR, int RULE, bool FQ>
 __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_amax_kernel(const QuantParams p, uint32_t* arrive,
-                                                                                uint32_t* status) {
+                                                                                uint32_t* status, uint32_t expected) {
     __shared__ float2 tab[128];
     __shared__ uint32_t red[kThreads / 32];
     __shared__ uint32_t go;
@@ -262,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_amax_kernel(c
         atomicAdd(arrive, 1u);
         uint32_t ok = 1;
         const unsigned long long t0 = clock64();
-        while (ld_acquire_u32(arrive) < gridDim.x) {
+        while (ld_acquire_u32(arrive) < expected) {
             if (clock64() - t0 > 4000000000ull) {
                 ok = 0;
                 if (status != nullptr) atomicOr(status, NVFP4_QUANT_TIMEOUT);

@@ -155,7 +155,8 @@ nvfp4_status launch_quant_amax(const nvfp4::QuantParams& p, uint32_t* arrive, ui
     // the resident CTAs (it fails instead of hanging if they do not fit)
     const dim3 grid = grouped_grid(static_cast<int64_t>(sm_count()) * ctas_per_sm<kernel>(), p.groups, p.gdiv.bpg);
     nvfp4::QuantParams pp = p;
-    void* args[] = {&pp, &arrive, &status};
+    uint32_t expected = grid.x;   // every CTA of the grid arrives at the barrier
+    void* args[] = {&pp, &arrive, &status, &expected};
     if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), grid, dim3(kThreads), args, 0, stream) !=
         cudaSuccess) {
         cudaGetLastError();   // refused (e.g. the grid cannot be resident): the caller runs two launches
