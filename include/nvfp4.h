@@ -43,9 +43,12 @@
  *
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller. The library allocates no
- *     memory, keeps no state between calls besides cached device attributes, and never
- *     synchronizes the host: work is enqueued on `stream` (0 = the legacy default stream) and
- *     completes in stream order.
+ *     memory and never synchronizes the host: work is enqueued on `stream` (0 = the legacy
+ *     default stream) and completes in stream order. Its only state between calls is a
+ *     per-device cache of device attributes (SM count, occupancies, the symbol address below,
+ *     the driver's tensor-map encoder) and one static device word per device: the grid-wide
+ *     barrier counter of nvfp4_amax_quantize / nvfp4_amax_fakequant calls made without a
+ *     workspace.
  *   - Shapes: groups >= 1, rows >= 0, cols >= 0 with cols % 16 == 0. An empty tensor
  *     (rows == 0 or cols == 0) is valid; each function states what it writes for one.
  *   - Alignment: BF16 tensors (x, y) 32 bytes, codes 8 bytes, choice/amax/tscale 4 bytes.
@@ -55,8 +58,9 @@
  *   - Errors: argument errors are detected on the host and returned before anything is
  *     enqueued (no output is touched). A launch failure returns NVFP4_ERR_CUDA. Kernels
  *     contain no device-side assert or trap. The only waits are the GEMM's mbarrier waits on
- *     its own copies and tensor-core work; each is bounded (about two seconds) and reports a
- *     timeout through the GEMM's status word.
+ *     its own copies and tensor-core work, and the grid-wide barrier of the one-launch amax +
+ *     quantize kernel (every CTA resident by a cooperative launch). Each is bounded (about two
+ *     seconds) and reports a timeout through the caller's status word.
  *   - Buffers must live on the device that is current for the calling thread.
  */
 #ifndef NVFP4_H
@@ -149,28 +153,44 @@ NVFP4_API nvfp4_status nvfp4_fakequant(const uint16_t* x, int64_t groups, int64_
                              uint16_t* y, uint8_t* choice, cudaStream_t stream);
 
 /* Bit set in a quantizer's status word when the grid-wide wait of nvfp4_amax_quantize or
- * nvfp4_amax_fakequant timed out (about two seconds); the outputs other than amax are then
- * not written. */
+ * nvfp4_amax_fakequant timed out (about two seconds) in at least one CTA. The outputs other
+ * than amax are then undefined: a CTA whose wait ran out writes nothing, but CTAs that saw
+ * the last arrival before their own limit go on and write their tiles, so the outputs may be
+ * partly written. */
 #define NVFP4_QUANT_TIMEOUT 2u
 
-/* nvfp4_amax followed by nvfp4_quantize in one launch: the dynamic tensor scale with the
- * fused amax ([FOS] Implementation details: the FP32 tensor scale comes from the tensor's
- * absolute maximum). Every CTA reduces max |x| over exactly the tiles it then quantizes,
- * all CTAs meet at a grid-wide barrier (a cooperative launch keeps them resident), and the
- * quantization re-reads the tiles, from L2 when the tensor fits there (126 MB). Outputs are
- * bit-identical to the two calls.
+/* nvfp4_amax followed by nvfp4_quantize in one launch, usable without any allocation. The
+ * pages have no counterpart for this entry point: it computes exactly what nvfp4_amax and
+ * nvfp4_quantize compute (outputs bit-identical to the two calls) and exists for callers that
+ * want one launch, or that cannot allocate device memory.
+ * Every CTA reduces max |x| over exactly the tiles it then quantizes, all CTAs meet at a
+ * grid-wide barrier (a cooperative launch keeps them resident), and the quantization re-reads
+ * the tiles, from L2 when the tensor fits there (126 MB). The barrier needs one 32-bit counter
+ * of scratch memory, whatever the tensor's shape.
  *   x, groups, rows, cols, mode, rule, codes, scales, tscale, choice as nvfp4_quantize (in/out)
  *   amax       [groups] float, 4-byte aligned: max |x| per group, written here          (out)
- *   workspace  NULL, or one 4-byte-aligned device word the call may use (zero-filled in
- *              stream order before the launch). With NULL the call uses one word of
- *              library memory per device and allocates nothing; such calls must not run
- *              concurrently on one device (different streams), while calls with their own
- *              workspaces may.                                                    (scratch)
+ *   workspace  NULL, or one 4-byte-aligned device word (the counter), zero-filled by the
+ *              call in stream order before the launch. With NULL the call allocates nothing:
+ *              it uses a static device word of the library (one per device that loads the
+ *              library, held until the process exits), for callers that cannot call
+ *              cudaMalloc: code running while a CUDA graph is being captured in the global
+ *              capture mode (where cudaMalloc is not allowed), serving runtimes that reserve
+ *              all device memory for their own pool up front, and plain C callers handed
+ *              device buffers with no allocator of their own. The first NULL-workspace call on
+ *              a device looks the word's device address up (cudaGetSymbolAddress, with that
+ *              device current) and caches it, so make that first call before any stream
+ *              capture. Every NULL-workspace call on a device shares the word (the call
+ *              zero-fills it first): such calls must not overlap on the GPU (different
+ *              streams), or their barriers race; calls with their own workspaces may overlap.
+ *              No shape is refused for lack of scratch: one word is all any call needs.
+ *                                                                                (scratch)
  *   status     NULL, or a device word; NVFP4_QUANT_TIMEOUT is or-ed in on a timed-out
  *              grid-wide wait                                                        (in/out)
  * Group layouts the grouped quantizer does not take (several groups whose block count is not
  * a multiple of 32), empty tensors, and devices that refuse the cooperative launch (the grid
- * cannot be resident at once) run as the two separate launches. Errors as nvfp4_quantize. */
+ * cannot be resident at once) run as the two separate launches (the counter is then not
+ * used). Errors as nvfp4_quantize; NVFP4_ERR_CUDA also when the static
+ * word's address cannot be obtained. */
 NVFP4_API nvfp4_status nvfp4_amax_quantize(const uint16_t* x, int64_t groups, int64_t rows, int64_t cols,
                                            nvfp4_mode mode, nvfp4_rule rule, float* amax, uint8_t* codes,
                                            uint8_t* scales, float* tscale, uint8_t* choice, uint32_t* workspace,

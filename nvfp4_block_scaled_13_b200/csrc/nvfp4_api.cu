@@ -144,9 +144,34 @@ nvfp4_status dispatch_quant(nvfp4_mode mode, nvfp4_rule rule, const nvfp4::Quant
 // Internal: a cooperative or cluster launch was refused, and the caller takes its other path.
 constexpr nvfp4_status NVFP4_ERR_UNSUPPORTED_LAUNCH = static_cast<nvfp4_status>(1000);
 
-// Barrier counter of nvfp4_amax_quantize / nvfp4_amax_fakequant calls without a workspace:
-// library memory (one per device), so those calls allocate nothing; they must not overlap.
-__device__ __align__(256) uint32_t g_amax_quant_scratch[64];
+// Scratch of nvfp4_amax_quantize / nvfp4_amax_fakequant calls made without a workspace: the
+// grid-wide barrier's arrival counter, one 32-bit word (the most any call needs, whatever the
+// tensor's size). A __device__ variable exists once on every device that loads the library and
+// lives until the process exits, so these calls allocate nothing; calls that use it must not
+// overlap on the GPU (they would share the counter).
+constexpr int kNoAllocScratchWords = 1;
+static __device__ __align__(256) uint32_t g_amax_quant_scratch[kNoAllocScratchWords];
+
+// Device address of g_amax_quant_scratch on the current device. In host code the symbol is a
+// host-side stand-in, not a device address, so it is looked up once per device (with that
+// device current: the first call on a device does it) and cached.
+nvfp4_status noalloc_scratch(uint32_t** out) {
+    static std::atomic<uintptr_t> addr[kMaxDevices];
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return NVFP4_ERR_CUDA;
+    uintptr_t a = dev < kMaxDevices ? addr[dev].load(std::memory_order_acquire) : 0;
+    if (a == 0) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_amax_quant_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return NVFP4_ERR_CUDA;
+        }
+        a = reinterpret_cast<uintptr_t>(p);
+        if (dev < kMaxDevices) addr[dev].store(a, std::memory_order_release);
+    }
+    *out = reinterpret_cast<uint32_t*>(a);
+    return NVFP4_OK;
+}
 
 template <bool FOUR, int RULE, bool FQ>
 nvfp4_status launch_quant_amax(const nvfp4::QuantParams& p, uint32_t* arrive, uint32_t* status, cudaStream_t stream) {
@@ -230,9 +255,10 @@ nvfp4_status amax_quant_impl(const uint16_t* x, int64_t groups, int64_t rows, in
         return fq ? nvfp4_fakequant(x, groups, rows, cols, amax, mode, rule, y, choice, stream)
                   : nvfp4_quantize(x, groups, rows, cols, amax, mode, rule, codes, scales, tscale, choice, stream);
     }
-    if (workspace == nullptr &&
-        cudaGetSymbolAddress(reinterpret_cast<void**>(&workspace), g_amax_quant_scratch) != cudaSuccess)
-        return NVFP4_ERR_CUDA;
+    if (workspace == nullptr) {
+        st = noalloc_scratch(&workspace);
+        if (st != NVFP4_OK) return st;
+    }
     if (cudaMemsetAsync(amax, 0, static_cast<size_t>(groups) * sizeof(float), stream) != cudaSuccess ||
         cudaMemsetAsync(workspace, 0, sizeof(uint32_t), stream) != cudaSuccess)
         return NVFP4_ERR_CUDA;
