@@ -9,10 +9,12 @@
 //  - block scales without a division: lo = RN(m * RN(RN(1/beta) (1 - 2^-20))) and
 //    hi = RN(m * RN(RN(1/beta) (1 + 2^-20))) bracket the exact quotient RN(m/beta), so when
 //    E4M3(lo) == E4M3(hi) the scale is proven; otherwise the quotient sits at the E4M3
-//    rounding boundary between the two codes, and one exact fused multiply-add decides;
-//  - the decode scale d = RN(f32(s) * alpha) and its reciprocal for every E4M3 code s come
-//    from a 128-entry table per group in shared memory (kernels whose CTAs work inside one
-//    group at a time), or are computed per block (the generic kernel);
+//    rounding boundary between the two codes, and one comparison of m with the group's
+//    threshold for the upper code decides (kernels with a shared-memory table), or one exact
+//    fused multiply-add (the generic kernel);
+//  - the decode scale d = RN(f32(s) * alpha) and its reciprocal for every E4M3 code s, and the
+//    thresholds, come from tables per group in shared memory (kernels whose CTAs work inside
+//    one group at a time), or are computed per block (the generic kernel);
 //  - packed .f32x2 arithmetic, three-input max, and 32-bit in-group indices.
 #pragma once
 
@@ -110,6 +112,31 @@ __device__ __forceinline__ GroupCtx make_group(float amax, float six_m) {
     return c;
 }
 
+// The smallest BF16 value m >= 0 with E4M3(RN(m / beta)) >= s, as binary32 (+inf when no
+// finite m reaches code s, or beta <= 0; 0 for s = 0). Code s is reached past the E4M3
+// rounding boundary M between codes s - 1 and s (their midpoint, at most 5 significant bits):
+// with ties going to the even code, E4M3(t) >= s iff t >= M (s even) or t > M (s odd).
+// For t = RN(m / beta): t >= M iff m / beta >= H, H the midpoint between M and the binary32
+// number below it (a quotient exactly at H rounds to M, whose significand is even), and t > M
+// iff m / beta > H', H' the midpoint between M and the binary32 number above it. beta * H is
+// exact in binary64 (24 + 26 significant bits), so the threshold is that product rounded up to
+// binary32 and then up to BF16 (the smallest BF16 value at or above it), one BF16 step higher
+// when the comparison is strict and the product is itself that BF16 value.
+__device__ __forceinline__ float e4m3_threshold(uint32_t s, float beta) {
+    if (s == 0u) return 0.0f;
+    if (s >= 127u || !(beta > 0.0f)) return __int_as_float(0x7F800000);
+    const float2 v = e4m3x2_to_float2((s - 1u) | (s << 8));
+    const float M = 0.5f * (v.x + v.y);
+    const bool odd = s & 1u;
+    const float nb = __uint_as_float(__float_as_uint(M) + (odd ? 1u : 0xFFFFFFFFu));
+    const double h = 0.5 * (static_cast<double>(M) + static_cast<double>(nb));
+    const double V = static_cast<double>(beta) * h;
+    const uint32_t b = __float_as_uint(__double2float_ru(V));
+    uint32_t t = (b + 0xFFFFu) & 0xFFFF0000u;
+    if (odd && static_cast<double>(__uint_as_float(t)) == V) t += 0x10000u;
+    return __uint_as_float(t);
+}
+
 // E4M3(RN(m / beta)) when the bracket gave adjacent codes s_lo < s_hi (the conversions of lo
 // and hi). The E4M3 rounding boundary M between them has at most 5 significant bits and
 // hi lies in [M, M (1 + 2^-19)], so M is hi truncated to 5 significant bits. With t =
@@ -135,11 +162,14 @@ __device__ __forceinline__ uint32_t scale_at_boundary(float m, float beta, float
 // saturates to 448 like the quotient it bounds. E4M3 rounding is monotone, so equal
 // conversions of lo and hi are the exact scale; different ones are adjacent codes (E4M3
 // boundaries lie at least 2^-4 apart, relatively), and scale_at_boundary decides between
-// them. For data on a coarse grid, such as BF16 block maxima over a simple tensor scale,
-// RN(m / beta) falls exactly on an E4M3 boundary for a few percent of the blocks. Outside the
-// factors' valid range the exact division decides.
+// them: with a threshold table (thr, see fill_scale_tables), the exact code is s_lo plus
+// [m >= threshold of s_lo + 1]; without one, scale_at_boundary. For data on a coarse grid,
+// such as BF16 block maxima over a tensor scale with a short binary expansion, RN(m / beta)
+// falls exactly on an E4M3 boundary for a few percent of the blocks, so most warps meet one:
+// the threshold comparison keeps that path to a few instructions. Outside the factors' valid
+// range the exact division decides.
 template <bool FOUR>
-__device__ __forceinline__ uint32_t block_scales(float m, const GroupCtx& c) {
+__device__ __forceinline__ uint32_t block_scales(float m, const GroupCtx& c, const float* thr = nullptr) {
     if (c.fast) {
         if (FOUR) {
             const float2 lo = mul2(make_float2(m, m), make_float2(c.yl6, c.yl4));
@@ -147,6 +177,11 @@ __device__ __forceinline__ uint32_t block_scales(float m, const GroupCtx& c) {
             const uint32_t wl = e4m3x2(lo.x, lo.y), wh = e4m3x2(hi.x, hi.y);
             if (wl == wh) return wl;
             uint32_t s6 = wl & 0xFFu, s4 = wl >> 8;
+            if (thr != nullptr) {
+                s6 += m >= thr[s6 + 1u] ? 1u : 0u;
+                s4 += m >= thr[128u + s4 + 1u] ? 1u : 0u;
+                return s6 | (s4 << 8);
+            }
             if (s6 != (wh & 0xFFu)) s6 = scale_at_boundary(m, c.beta6, hi.x, s6, wh & 0xFFu);
             if (s4 != (wh >> 8)) s4 = scale_at_boundary(m, c.beta4, hi.y, s4, wh >> 8);
             return s6 | (s4 << 8);
@@ -154,6 +189,7 @@ __device__ __forceinline__ uint32_t block_scales(float m, const GroupCtx& c) {
             const float2 b = mul2(make_float2(m, m), make_float2(c.yl6, c.yh6));
             const uint32_t b6 = e4m3x2(b.x, b.y);
             if ((b6 & 0xFFu) == (b6 >> 8)) return b6 & 0xFFu;
+            if (thr != nullptr) return (b6 & 0xFFu) + (m >= thr[(b6 & 0xFFu) + 1u] ? 1u : 0u);
             return scale_at_boundary(m, c.beta6, b.y, b6 & 0xFFu, b6 >> 8);
         }
     }
@@ -166,6 +202,21 @@ __device__ __forceinline__ uint32_t block_scales(float m, const GroupCtx& c) {
 __device__ __forceinline__ float2 scale_entry(uint32_t s, float alpha) {
     const float d = __fmul_rn(e4m3x2_to_float2(s).x, alpha);
     return make_float2(d, recip_clamped(d));
+}
+
+// Per-group tables in shared memory (256 float2 = 2 KiB), built by the first 256 threads of a
+// CTA: entries 0-127, (d, 1/d) by E4M3 code (code 127, not produced, repeats 126); then, as
+// floats, the thresholds e4m3_threshold(s, beta_6) for s = 0..127 and (Four Over Six) those
+// for beta_4. The thresholds are only built, and only read, when the bracket is in use.
+template <bool FOUR>
+__device__ __forceinline__ void fill_scale_tables(float2* tab, const GroupCtx& gc, uint32_t tid) {
+    if (tid < 128u) {
+        tab[tid] = scale_entry(tid == 127u ? 126u : tid, gc.alpha);
+    } else if (tid < 256u && gc.fast) {
+        float* thr = reinterpret_cast<float*>(tab + 128);
+        thr[tid - 128u] = e4m3_threshold(tid - 128u, gc.beta6);
+        if (FOUR) thr[tid] = e4m3_threshold(tid - 128u, gc.beta4);
+    }
 }
 
 // One candidate (target maximum K) of one block: its codes, their exact values as f16x2
@@ -201,7 +252,7 @@ __device__ __forceinline__ float candidate(const float2 (&x)[8], float r, float 
 // Quantize the block in `w` (eight BF16 pairs) into registers: the kept candidate's codes
 // (clo: elements 0-7, chi: 8-15, element 2j in the low nibble), its E4M3 scale s and decode
 // scale d, and (FQ) its values as f16x2 words in h. Returns whether target 4 was kept.
-// TABLE: d and 1/d come from `tab`.
+// TABLE: d, 1/d and the scale thresholds come from `tab` (fill_scale_tables).
 template <bool FOUR, int RULE, bool FQ, bool TABLE>
 __device__ __forceinline__ bool quantize_block_regs(const uint32_t (&w)[8], const GroupCtx& gc, const float2* tab,
                                                     uint32_t& clo, uint32_t& chi, uint32_t& s, float& dsel,
@@ -217,7 +268,7 @@ __device__ __forceinline__ bool quantize_block_regs(const uint32_t (&w)[8], cons
     const float m05 = max3(fabsf(x[5].y), fabsf(x[6].x), fabsf(x[6].y));
     const float m06 = max3(fabsf(x[7].x), fabsf(x[7].y), 0.0f);
     const float m = fmaxf(max3(m01, m02, m03), max3(m04, m05, m06));
-    const uint32_t s2 = block_scales<FOUR>(m, gc);
+    const uint32_t s2 = block_scales<FOUR>(m, gc, TABLE ? reinterpret_cast<const float*>(tab + 128) : nullptr);
     const uint32_t i6 = __byte_perm(s2, 0u, 0x4440), i4 = __byte_perm(s2, 0u, 0x4441);
     const float2 e6 = TABLE ? tab[i6] : scale_entry(i6, gc.alpha);
     const float err6 = candidate<RULE>(x, e6.y, e6.x, clo, chi, h);

@@ -389,7 +389,7 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
         acc_empty, drain;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile uint32_t stop_sh;
-    __shared__ float2 tab[128];
+    __shared__ float2 tab[256];   // the prologue's scale tables (fill_scale_tables)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t n_ct = p.k / 64;                   // scale tiles per 128 rows
     const int nk = static_cast<int>(p.k / kBK);
@@ -424,7 +424,7 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
     if (QUANT) {
         constexpr float kSixM = FOUR ? 1536.0f : 2688.0f;
         gc = make_group<FOUR>(__ldg(p.x_amax), kSixM);
-        if (tid < 128) tab[tid] = scale_entry(tid == 127 ? 126u : static_cast<uint32_t>(tid), gc.alpha);
+        fill_scale_tables<FOUR>(tab, gc, static_cast<uint32_t>(tid));
     }
     tc_fence_before();
     __syncthreads();

@@ -129,7 +129,7 @@ __device__ __forceinline__ void quant_segment(const QuantParams& p, float2* tab,
     if (tile < tend) load_tile(xg, tile, lane, bpg, a0, a1);   // in flight while the table is built
     const GroupCtx gc = make_group<FOUR>(FRESH ? ld_acquire_f32(p.amax + g) : __ldg(p.amax + g), kSixM);
     __syncthreads();                       // the previous group's table is no longer read
-    if (threadIdx.x < 128) tab[threadIdx.x] = scale_entry(threadIdx.x == 127 ? 126u : threadIdx.x, gc.alpha);
+    fill_scale_tables<FOUR>(tab, gc, threadIdx.x);
     if (!FQ && write_tscale && threadIdx.x == 0) p.tscale[g] = gc.alpha;
     __syncthreads();
     uint8_t* cg = FQ ? nullptr : p.codes + base * 8;
@@ -170,7 +170,7 @@ __device__ __forceinline__ void quant_segment(const QuantParams& p, float2* tab,
 // so every CTA slot works and the ranges differ by at most one tile.
 template <bool FOUR, int RULE, bool FQ, bool SWZ = false>
 __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kernel(const QuantParams p) {
-    __shared__ float2 tab[128];
+    __shared__ float2 tab[256];   // scale tables (fill_scale_tables)
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t bpg = static_cast<uint32_t>(p.gdiv.bpg);
     const uint32_t ntiles = (bpg + 63u) >> 6;
@@ -236,7 +236,7 @@ __device__ __forceinline__ void cta_max_to(uint32_t* red, uint32_t v, float* out
 template <bool FOUR, int RULE, bool FQ>
 __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_amax_kernel(const QuantParams p, uint32_t* arrive,
                                                                                 uint32_t* status, uint32_t expected) {
-    __shared__ float2 tab[128];
+    __shared__ float2 tab[256];   // scale tables (fill_scale_tables)
     __shared__ uint32_t red[kThreads / 32];
     __shared__ uint32_t go;
     const uint32_t lane = threadIdx.x & 31u;

@@ -2,7 +2,9 @@
 //
 // Conversions use the Blackwell cvt family ("Four Over Six ...", Implementation details:
 // the kernel is built on cvt instructions): f32 -> E2M1 pairs and f32 -> E4M3 pairs with
-// round-to-nearest-even and satfinite, and the exact widening conversions back to f16.
+// round-to-nearest-even and satfinite, and the exact widening conversions back to f16. f16 and
+// BF16 values are widened to binary32 by mixed-precision additions (sm_100), which run on the
+// FMA pipes: in the quantizer the ALU pipe is the busier one.
 // Arithmetic that decides a code or a choice is IEEE binary32 round-to-nearest; the packed
 // .f32x2 forms are lane-wise IEEE (sm_100+), so they give the same bits as scalar code.
 #pragma once
@@ -138,9 +140,15 @@ __device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t& h0, uint32
         : "r"(w));
 }
 
+// f16 pair -> two binary32 (exact): each half widened by a mixed-precision addition of -0
+// (f16 + f32 -> f32), which runs on the FMA pipes and leaves the ALU to the conversions.
 __device__ __forceinline__ float2 f16x2_to_float2(uint32_t h) {
-    __half2 v = *reinterpret_cast<__half2*>(&h);
-    return __half22float2(v);
+    float2 r;
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "add.rn.f32.f16 %0, a, 0f80000000;\n\tadd.rn.f32.f16 %1, b, 0f80000000;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "r"(h));
+    return r;
 }
 
 // Two non-negative binary32 values -> two E4M3 bytes (round to nearest even, satfinite):
@@ -165,9 +173,15 @@ __device__ __forceinline__ uint32_t bf16x2(float2 v) {
     return *reinterpret_cast<uint32_t*>(&b);
 }
 
-// BF16x2 bits -> two binary32 (exact).
+// BF16x2 bits -> two binary32 (exact), by mixed-precision additions of -0 like f16x2_to_float2
+// (x + -0 is x for every finite x, zeros keep their sign).
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
-    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    float2 r;
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "add.rn.f32.bf16 %0, a, 0f80000000;\n\tadd.rn.f32.bf16 %1, b, 0f80000000;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "r"(w));
+    return r;
 }
 
 }  // namespace nvfp4
