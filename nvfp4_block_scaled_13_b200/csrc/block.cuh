@@ -48,6 +48,7 @@ struct GroupDiv {
 };
 
 struct QuantParams {
+    uint32_t ident = 0x3210u;   // identity byte selector, passed at run time (e2m1x8_and_decode)
     const uint16_t* x;
     const float* amax;
     uint8_t* codes;      // codes output (quantize) or nullptr (fake-quant)
@@ -93,11 +94,13 @@ __device__ __forceinline__ float recip_clamped(float d) {
 struct GroupCtx {
     float alpha, beta6, beta4, yl6, yh6, yl4, yh4;
     bool fast;
+    uint32_t ident;   // the kernel argument's identity byte selector (e2m1x8_and_decode)
 };
 
 template <bool FOUR>
-__device__ __forceinline__ GroupCtx make_group(float amax, float six_m) {
+__device__ __forceinline__ GroupCtx make_group(float amax, float six_m, uint32_t ident) {
     GroupCtx c;
+    c.ident = ident;
     c.alpha = __fdiv_rn(amax, six_m);
     c.beta6 = __fmul_rn(6.0f, c.alpha);
     c.beta4 = __fmul_rn(4.0f, c.alpha);
@@ -225,13 +228,13 @@ __device__ __forceinline__ void fill_scale_tables(float2* tab, const GroupCtx& g
 // element indices (for MSE the two lanes of a packed pair), added at the end.
 template <int RULE>
 __device__ __forceinline__ float candidate(const float2 (&x)[8], float r, float d, uint32_t& c_lo,
-                                           uint32_t& c_hi, uint32_t (&h)[8]) {
+                                           uint32_t& c_hi, uint32_t (&h)[8], uint32_t ident) {
     const float2 rr = make_float2(r, r), nd = make_float2(-d, -d);
     float2 y[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) y[j] = mul2(x[j], rr);
-    c_lo = e2m1x8_and_decode(y[0], y[1], y[2], y[3], h[0], h[1], h[2], h[3]);
-    c_hi = e2m1x8_and_decode(y[4], y[5], y[6], y[7], h[4], h[5], h[6], h[7]);
+    c_lo = e2m1x8_and_decode(y[0], y[1], y[2], y[3], h[0], h[1], h[2], h[3], ident);
+    c_hi = e2m1x8_and_decode(y[4], y[5], y[6], y[7], h[4], h[5], h[6], h[7], ident);
     float2 acc = make_float2(0.0f, 0.0f);
     float emax = 0.0f;
 #pragma unroll
@@ -260,25 +263,24 @@ __device__ __forceinline__ bool quantize_block_regs(const uint32_t (&w)[8], cons
     float2 x[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) x[j] = unpack_bf16x2(w[j]);
-    // max over {0, |x_i|}: depth-3 tree of 3-input max (the same value as a running max)
-    const float m01 = max3(0.0f, fabsf(x[0].x), fabsf(x[0].y));
-    const float m02 = max3(fabsf(x[1].x), fabsf(x[1].y), fabsf(x[2].x));
-    const float m03 = max3(fabsf(x[2].y), fabsf(x[3].x), fabsf(x[3].y));
-    const float m04 = max3(fabsf(x[4].x), fabsf(x[4].y), fabsf(x[5].x));
-    const float m05 = max3(fabsf(x[5].y), fabsf(x[6].x), fabsf(x[6].y));
-    const float m06 = max3(fabsf(x[7].x), fabsf(x[7].y), 0.0f);
-    const float m = fmaxf(max3(m01, m02, m03), max3(m04, m05, m06));
+    // max of the 16 |x_i|: a depth-3 tree of 3-input max (the same value as a running max)
+    const float m01 = max3(fabsf(x[0].x), fabsf(x[0].y), fabsf(x[1].x));
+    const float m02 = max3(fabsf(x[1].y), fabsf(x[2].x), fabsf(x[2].y));
+    const float m03 = max3(fabsf(x[3].x), fabsf(x[3].y), fabsf(x[4].x));
+    const float m04 = max3(fabsf(x[4].y), fabsf(x[5].x), fabsf(x[5].y));
+    const float m05 = max3(fabsf(x[6].x), fabsf(x[6].y), fabsf(x[7].x));
+    const float m = fmaxf(max3(m01, m02, m03), max3(m04, m05, fabsf(x[7].y)));
     const uint32_t s2 = block_scales<FOUR>(m, gc, TABLE ? reinterpret_cast<const float*>(tab + 128) : nullptr);
     const uint32_t i6 = __byte_perm(s2, 0u, 0x4440), i4 = __byte_perm(s2, 0u, 0x4441);
     const float2 e6 = TABLE ? tab[i6] : scale_entry(i6, gc.alpha);
-    const float err6 = candidate<RULE>(x, e6.y, e6.x, clo, chi, h);
+    const float err6 = candidate<RULE>(x, e6.y, e6.x, clo, chi, h, gc.ident);
     s = i6;
     dsel = e6.x;
     bool four = false;
     if (FOUR) {
         const float2 e4 = TABLE ? tab[i4] : scale_entry(i4, gc.alpha);
         uint32_t c4lo, c4hi, h4[8];
-        const float err4 = candidate<RULE>(x, e4.y, e4.x, c4lo, c4hi, h4);
+        const float err4 = candidate<RULE>(x, e4.y, e4.x, c4lo, c4hi, h4, gc.ident);
         four = err4 < err6;   // ties keep target 6
         if (four) {
             clo = c4lo;

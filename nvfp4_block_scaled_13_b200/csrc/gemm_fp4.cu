@@ -343,6 +343,7 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
 namespace {
 
 struct GemmParams {
+    uint32_t ident = 0x3210u;  // prologue variant: identity byte selector (e2m1x8_and_decode)
     const uint16_t* x;        // prologue variant: BF16 activations [m, k] (32-byte aligned)
     const float* x_amax;      // prologue variant: amax of x, [1]
     const uint8_t* x_scales;  // pre-quantized variant: tiled scales of x
@@ -423,7 +424,7 @@ __global__ void __launch_bounds__(gemm_threads<QUANT>(), 1)
     GroupCtx gc{};
     if (QUANT) {
         constexpr float kSixM = FOUR ? 1536.0f : 2688.0f;
-        gc = make_group<FOUR>(__ldg(p.x_amax), kSixM);
+        gc = make_group<FOUR>(__ldg(p.x_amax), kSixM, p.ident);
         fill_scale_tables<FOUR>(tab, gc, static_cast<uint32_t>(tid));
     }
     tc_fence_before();

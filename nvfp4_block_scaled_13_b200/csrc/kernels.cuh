@@ -127,7 +127,7 @@ __device__ __forceinline__ void quant_segment(const QuantParams& p, float2* tab,
     const uint16_t* xg = p.x + base * 16;
     uint32_t a0[8], a1[8];
     if (tile < tend) load_tile(xg, tile, lane, bpg, a0, a1);   // in flight while the table is built
-    const GroupCtx gc = make_group<FOUR>(FRESH ? ld_acquire_f32(p.amax + g) : __ldg(p.amax + g), kSixM);
+    const GroupCtx gc = make_group<FOUR>(FRESH ? ld_acquire_f32(p.amax + g) : __ldg(p.amax + g), kSixM, p.ident);
     __syncthreads();                       // the previous group's table is no longer read
     fill_scale_tables<FOUR>(tab, gc, threadIdx.x);
     if (!FQ && write_tscale && threadIdx.x == 0) p.tscale[g] = gc.alpha;
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantParams p)
                 const int64_t g = p.gdiv(b);
                 const int64_t g_start = g * p.gdiv.bpg;
                 g_end = g_start + p.gdiv.bpg;
-                gc = make_group<FOUR>(__ldg(p.amax + g), kSixM);
+                gc = make_group<FOUR>(__ldg(p.amax + g), kSixM, p.ident);
                 if (!FQ && b == g_start) p.tscale[g] = gc.alpha;
             }
             four = quantize_block<FOUR, RULE, FQ, false>(cur, gc, nullptr, FQ ? nullptr : p.codes + b * 8,

@@ -101,31 +101,6 @@ __device__ __forceinline__ float ld_acquire_f32(const float* p) {
 
 // ---- format conversions ------------------------------------------------------------------
 
-// Eight binary32 values (four pairs p[j] = (element 2j, element 2j+1)) -> eight E2M1 codes
-// packed so that element k sits in bits [4k, 4k+4) (the low nibble of each byte holds the
-// even element; cvt ... d, a, b puts a in the high nibble and b in the low nibble), and the
-// codes' exact values as four f16x2 words (word j: element 2j low, 2j+1 high).
-// The decode reads the .b8 results of the conversions inside the same asm block: decoding
-// bytes that were first packed into a 32-bit word and unpacked again gave zeros for bytes 2
-// and 3 on sm_100a, so this pattern is avoided.
-__device__ __forceinline__ uint32_t e2m1x8_and_decode(float2 p0, float2 p1, float2 p2, float2 p3, uint32_t& h0,
-                                                      uint32_t& h1, uint32_t& h2, uint32_t& h3) {
-    uint32_t r;
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, %6, %5;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, %8, %7;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b2, %10, %9;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b3, %12, %11;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %1, b0;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %2, b1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %3, b2;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %4, b3;\n\t"
-        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-        : "=r"(r), "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
-        : "f"(p0.x), "f"(p0.y), "f"(p1.x), "f"(p1.y), "f"(p2.x), "f"(p2.y), "f"(p3.x), "f"(p3.y));
-    return r;
-}
-
 // Eight packed E2M1 codes loaded from memory -> four f16x2 words (exact); word j holds
 // elements 2j (low half) and 2j+1 (high half).
 __device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t& h0, uint32_t& h1, uint32_t& h2,
@@ -138,6 +113,32 @@ __device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t& h0, uint32
         "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
         : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
         : "r"(w));
+}
+
+// Eight binary32 values (four pairs p[j] = (element 2j, element 2j+1)) -> eight E2M1 codes
+// packed so that element k sits in bits [4k, 4k+4) (the low nibble of each byte holds the
+// even element; cvt ... d, a, b puts a in the high nibble and b in the low nibble), and the
+// codes' exact values as four f16x2 words (word j: element 2j low, 2j+1 high).
+// The four conversions write their bytes straight into the packed word; the decode then reads
+// the word's bytes. The word passes through a byte permutation whose selector is the identity
+// 0x3210 given at run time (`ident`, a kernel argument), so the compiler treats it as an
+// arbitrary word: letting the compiler forward the conversions' bytes into the decode
+// instead (the same code without the permutation) decoded bytes 2 and 3 as zeros with CUDA
+// 12.9 for sm_100a, and decoding each byte before packing costs about three more
+// instructions per word.
+__device__ __forceinline__ uint32_t e2m1x8_and_decode(float2 p0, float2 p1, float2 p2, float2 p3, uint32_t& h0,
+                                                      uint32_t& h1, uint32_t& h2, uint32_t& h3, uint32_t ident) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(p0.x), "f"(p0.y), "f"(p1.x), "f"(p1.y), "f"(p2.x), "f"(p2.y), "f"(p3.x), "f"(p3.y));
+    e2m1x8_to_f16x2(__byte_perm(r, 0u, ident), h0, h1, h2, h3);
+    return r;
 }
 
 // f16 pair -> two binary32 (exact): each half widened by a mixed-precision addition of -0
