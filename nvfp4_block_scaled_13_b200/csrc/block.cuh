@@ -95,6 +95,7 @@ struct GroupCtx {
     float alpha, beta6, beta4, yl6, yh6, yl4, yh4;
     bool fast;
     uint32_t ident;   // the kernel argument's identity byte selector (e2m1x8_and_decode)
+    uint32_t lane8, dtab;   // decode table (candidate_tab): lane * 8 and the table's shared address
 };
 
 template <bool FOUR>
@@ -252,11 +253,59 @@ __device__ __forceinline__ float candidate(const float2 (&x)[8], float r, float 
     return RULE == kMaxErr ? emax : __fadd_rn(acc.x, acc.y);
 }
 
+// Decode table in shared memory (dynamic, kDecodeTableBytes = 64 KiB): for every E2M1 byte e
+// (two codes) the binary32 values of both codes, in 32 copies at e * 256 + lane * 8, so that
+// the 16 lanes of a shared-memory phase each read their own bank pair whatever bytes they look
+// up. One byte permutation forms a lookup's address: the code byte into bits 8-15 and
+// lane * 8 into bits 0-7. The values are the hardware decode's (cvt.rn.f16x2.e2m1x2, widened).
+constexpr uint32_t kDecodeTableBytes = 65536;
+
+__device__ __forceinline__ void fill_decode_table(float2* dect) {
+    for (uint32_t i = threadIdx.x; i < 8192u; i += blockDim.x) {
+        uint32_t h0, h1, h2, h3;
+        e2m1x8_to_f16x2(i >> 5, h0, h1, h2, h3);
+        dect[i] = f16x2_to_float2(h0);
+    }
+}
+
+// candidate() with the code values read from the decode table instead of decoded and widened:
+// per pair of elements one byte permutation and one 8-byte shared-memory load replace a decode,
+// its byte extraction and two widening additions (about 2 instructions fewer per pair, and
+// the ALU and FMA pipes lose work to the load pipe). Same values, same error, bit for bit.
+template <int RULE>
+__device__ __forceinline__ float candidate_tab(const float2 (&x)[8], float r, float d, uint32_t& c_lo,
+                                               uint32_t& c_hi, uint32_t lane8, uint32_t dtab) {
+    const float2 rr = make_float2(r, r), nd = make_float2(-d, -d);
+    float2 y[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = mul2(x[j], rr);
+    c_lo = e2m1x8(y[0], y[1], y[2], y[3]);
+    c_hi = e2m1x8(y[4], y[5], y[6], y[7]);
+    float2 acc = make_float2(0.0f, 0.0f);
+    float emax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t w = j < 4 ? c_lo : c_hi;
+        const float2 v = lds_f2(dtab + __byte_perm(w, lane8, 0x5504u | ((j & 3) << 4)));
+        const float2 e = fma2(v, nd, x[j]);
+        if (RULE == kMse) {
+            acc = fma2(e, e, acc);
+        } else if (RULE == kMae) {
+            acc.x = __fadd_rn(acc.x, fabsf(e.x));
+            acc.y = __fadd_rn(acc.y, fabsf(e.y));
+        } else {
+            emax = max3(emax, fabsf(e.x), fabsf(e.y));
+        }
+    }
+    return RULE == kMaxErr ? emax : __fadd_rn(acc.x, acc.y);
+}
+
 // Quantize the block in `w` (eight BF16 pairs) into registers: the kept candidate's codes
 // (clo: elements 0-7, chi: 8-15, element 2j in the low nibble), its E4M3 scale s and decode
 // scale d, and (FQ) its values as f16x2 words in h. Returns whether target 4 was kept.
-// TABLE: d, 1/d and the scale thresholds come from `tab` (fill_scale_tables).
-template <bool FOUR, int RULE, bool FQ, bool TABLE>
+// TABLE: d, 1/d and the scale thresholds come from `tab` (fill_scale_tables). DEC: code values
+// come from the decode table (gc.dtab; not with FQ, which keeps the decoded words).
+template <bool FOUR, int RULE, bool FQ, bool TABLE, bool DEC = false>
 __device__ __forceinline__ bool quantize_block_regs(const uint32_t (&w)[8], const GroupCtx& gc, const float2* tab,
                                                     uint32_t& clo, uint32_t& chi, uint32_t& s, float& dsel,
                                                     uint32_t (&h)[8]) {
@@ -273,14 +322,16 @@ __device__ __forceinline__ bool quantize_block_regs(const uint32_t (&w)[8], cons
     const uint32_t s2 = block_scales<FOUR>(m, gc, TABLE ? reinterpret_cast<const float*>(tab + 128) : nullptr);
     const uint32_t i6 = __byte_perm(s2, 0u, 0x4440), i4 = __byte_perm(s2, 0u, 0x4441);
     const float2 e6 = TABLE ? tab[i6] : scale_entry(i6, gc.alpha);
-    const float err6 = candidate<RULE>(x, e6.y, e6.x, clo, chi, h, gc.ident);
+    const float err6 = DEC ? candidate_tab<RULE>(x, e6.y, e6.x, clo, chi, gc.lane8, gc.dtab)
+                           : candidate<RULE>(x, e6.y, e6.x, clo, chi, h, gc.ident);
     s = i6;
     dsel = e6.x;
     bool four = false;
     if (FOUR) {
         const float2 e4 = TABLE ? tab[i4] : scale_entry(i4, gc.alpha);
         uint32_t c4lo, c4hi, h4[8];
-        const float err4 = candidate<RULE>(x, e4.y, e4.x, c4lo, c4hi, h4, gc.ident);
+        const float err4 = DEC ? candidate_tab<RULE>(x, e4.y, e4.x, c4lo, c4hi, gc.lane8, gc.dtab)
+                               : candidate<RULE>(x, e4.y, e4.x, c4lo, c4hi, h4, gc.ident);
         four = err4 < err6;   // ties keep target 6
         if (four) {
             clo = c4lo;
@@ -299,12 +350,12 @@ __device__ __forceinline__ bool quantize_block_regs(const uint32_t (&w)[8], cons
 // Quantize the block in `w` and store its codes + scale (or fake-quant BF16); returns whether
 // target 4 was kept. ok = false (a lane past the end of the group) computes but stores nothing
 // and returns false.
-template <bool FOUR, int RULE, bool FQ, bool TABLE>
+template <bool FOUR, int RULE, bool FQ, bool TABLE, bool DEC = false>
 __device__ __forceinline__ bool quantize_block(const uint32_t (&w)[8], const GroupCtx& gc, const float2* tab,
                                                uint8_t* codes8, uint8_t* scale1, uint16_t* y16, bool ok = true) {
     uint32_t clo, chi, s, h[8];
     float dsel;
-    const bool four = quantize_block_regs<FOUR, RULE, FQ, TABLE>(w, gc, tab, clo, chi, s, dsel, h);
+    const bool four = quantize_block_regs<FOUR, RULE, FQ, TABLE, DEC>(w, gc, tab, clo, chi, s, dsel, h);
     if (FQ) {   // q = RN(v * d) of the kept candidate, rounded to BF16
         const float2 dd = make_float2(dsel, dsel);
         uint32_t out[8];

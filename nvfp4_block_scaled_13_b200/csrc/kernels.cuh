@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
 // blocks_per_group % 32 == 0) and blocks_per_group < 2^30.
 // SWZ: scales go to the tiled GEMM layout (one group only).
 // One warp tile (64 blocks) of one group; lane t works on blocks 64 tile + t and + 32.
-template <bool FOUR, int RULE, bool FQ, bool SWZ>
+template <bool FOUR, int RULE, bool FQ, bool SWZ, bool DEC = false>
 __device__ __forceinline__ void quant_tile(const QuantParams& p, const GroupCtx& gc, const float2* tab,
                                            uint32_t tile, uint32_t lane, uint32_t bpg, uint8_t* cg, uint8_t* sg,
                                            uint16_t* yg, uint32_t* chw, int64_t base,
@@ -87,9 +87,9 @@ __device__ __forceinline__ void quant_tile(const QuantParams& p, const GroupCtx&
     uint8_t* c0 = FQ ? nullptr : cg + static_cast<size_t>(a) * 8;
     uint8_t* s0 = FQ ? nullptr : sg + a;
     uint16_t* y0 = FQ ? yg + static_cast<size_t>(a) * 16 : nullptr;
-    const bool fa = quantize_block<FOUR, RULE, FQ, true>(ca, gc, tab, c0, SWZ ? p.scales + tiled_scale_offset(a, p) : s0,
+    const bool fa = quantize_block<FOUR, RULE, FQ, true, DEC>(ca, gc, tab, c0, SWZ ? p.scales + tiled_scale_offset(a, p) : s0,
                                                          y0, oka);
-    const bool fb = quantize_block<FOUR, RULE, FQ, true>(cb, gc, tab, FQ ? nullptr : c0 + 256,
+    const bool fb = quantize_block<FOUR, RULE, FQ, true, DEC>(cb, gc, tab, FQ ? nullptr : c0 + 256,
                                                          SWZ ? p.scales + tiled_scale_offset(a + 32u, p) : (FQ ? nullptr : s0 + 32),
                                                          FQ ? y0 + 512 : nullptr, okb);
     if (p.choice != nullptr) {
@@ -118,16 +118,19 @@ __device__ __forceinline__ void load_tile(const uint16_t* xg, uint32_t tile, uin
 // stores the group's tensor scale.
 // FRESH: the amax was written during this launch (by other CTAs), so it is read with a
 // gpu-scope acquire load rather than through the read-only cache.
-template <bool FOUR, int RULE, bool FQ, bool SWZ, bool FRESH = false>
+template <bool FOUR, int RULE, bool FQ, bool SWZ, bool FRESH = false, bool DEC = false>
 __device__ __forceinline__ void quant_segment(const QuantParams& p, float2* tab, int64_t g, uint32_t tile,
-                                              uint32_t tend, uint32_t stride, uint32_t lane, bool write_tscale) {
+                                              uint32_t tend, uint32_t stride, uint32_t lane, bool write_tscale,
+                                              uint32_t dtab = 0) {
     constexpr float kSixM = FOUR ? 1536.0f : 2688.0f;   // 6 * 256 or 6 * 448
     const uint32_t bpg = static_cast<uint32_t>(p.gdiv.bpg);
     const int64_t base = g * static_cast<int64_t>(bpg);
     const uint16_t* xg = p.x + base * 16;
     uint32_t a0[8], a1[8];
     if (tile < tend) load_tile(xg, tile, lane, bpg, a0, a1);   // in flight while the table is built
-    const GroupCtx gc = make_group<FOUR>(FRESH ? ld_acquire_f32(p.amax + g) : __ldg(p.amax + g), kSixM, p.ident);
+    GroupCtx gc = make_group<FOUR>(FRESH ? ld_acquire_f32(p.amax + g) : __ldg(p.amax + g), kSixM, p.ident);
+    gc.lane8 = lane * 8u;
+    gc.dtab = dtab;
     __syncthreads();                       // the previous group's table is no longer read
     fill_scale_tables<FOUR>(tab, gc, threadIdx.x);
     if (!FQ && write_tscale && threadIdx.x == 0) p.tscale[g] = gc.alpha;
@@ -145,19 +148,19 @@ __device__ __forceinline__ void quant_segment(const QuantParams& p, float2* tab,
                 b1[k] = a1[k];
             }
             if (tile + stride < tend) load_tile(xg, tile + stride, lane, bpg, a0, a1);
-            quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, base, b0, b1);
+            quant_tile<FOUR, RULE, FQ, SWZ, DEC>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, base, b0, b1);
         }
     } else {
         uint32_t b0[8], b1[8];
         while (tile < tend) {
             uint32_t nt = tile + stride;
             if (nt < tend) load_tile(xg, nt, lane, bpg, b0, b1);
-            quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, base, a0, a1);
+            quant_tile<FOUR, RULE, FQ, SWZ, DEC>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, base, a0, a1);
             tile = nt;
             if (tile >= tend) break;
             nt = tile + stride;
             if (nt < tend) load_tile(xg, nt, lane, bpg, a0, a1);
-            quant_tile<FOUR, RULE, FQ, SWZ>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, base, b0, b1);
+            quant_tile<FOUR, RULE, FQ, SWZ, DEC>(p, gc, tab, tile, lane, bpg, cg, sg, yg, chw, base, b0, b1);
             tile = nt;
         }
     }
@@ -171,6 +174,10 @@ __device__ __forceinline__ void quant_segment(const QuantParams& p, float2* tab,
 template <bool FOUR, int RULE, bool FQ, bool SWZ = false>
 __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kernel(const QuantParams p) {
     __shared__ float2 tab[256];   // scale tables (fill_scale_tables)
+    extern __shared__ __align__(16) float2 dect[];   // decode table (Four Over Six codes): 64 KiB dynamic
+    constexpr bool kDec = FOUR && !FQ;
+    if (kDec) fill_decode_table(dect);
+    const uint32_t dtab = kDec ? smem_addr(dect) : 0u;
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t bpg = static_cast<uint32_t>(p.gdiv.bpg);
     const uint32_t ntiles = (bpg + 63u) >> 6;
@@ -186,7 +193,8 @@ __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kerne
         const int64_t g = t / ntiles;
         const uint32_t t0 = static_cast<uint32_t>(t - g * ntiles);
         const uint32_t t1 = static_cast<uint32_t>(min(end - g * ntiles, static_cast<int64_t>(ntiles)));
-        quant_segment<FOUR, RULE, FQ, SWZ>(p, tab, g, t0 + first, t1, stride, lane, one ? blockIdx.x == 0 : t0 == 0);
+        quant_segment<FOUR, RULE, FQ, SWZ, false, kDec>(p, tab, g, t0 + first, t1, stride, lane,
+                                                        one ? blockIdx.x == 0 : t0 == 0, dtab);
         t = g * ntiles + t1;
     }
 }

@@ -1,6 +1,7 @@
 // nvfp4_api.cu — the C ABI declared in include/nvfp4.h: argument validation, launch
 // configuration and kernel dispatch. No allocation, no host synchronization, no state
-// beyond a per-device cache of launch limits.
+// beyond a per-device cache of launch limits (and of the dynamic shared-memory allowance set
+// once per device for the kernels that hold the 64 KiB decode table).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -43,16 +44,38 @@ int sm_count() {
 // argument so that every kernel gets its own cache: the quantizer's instantiations share one
 // function type, and a cache keyed by the type would hand one kernel's occupancy to another.
 template <auto kernel>
-int ctas_per_sm() {
+int ctas_per_sm(size_t dyn_smem = 0) {
     static std::atomic<int> cache[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
     int v = (dev >= 0 && dev < kMaxDevices) ? cache[dev].load(std::memory_order_relaxed) : 0;
     if (v == 0) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kernel, kThreads, 0) != cudaSuccess || v <= 0) v = 1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kernel, kThreads, dyn_smem) != cudaSuccess || v <= 0)
+            v = 1;
         if (dev >= 0 && dev < kMaxDevices) cache[dev].store(v, std::memory_order_relaxed);
     }
     return v;
+}
+
+// Dynamic shared memory of the grouped quantizer: the decode table for Four Over Six codes.
+template <bool FOUR, bool FQ>
+constexpr size_t quant_dyn_smem() { return (FOUR && !FQ) ? nvfp4::kDecodeTableBytes : 0; }
+
+// Lets `kernel` use `bytes` of dynamic shared memory on the current device (set once per device).
+template <auto kernel>
+bool allow_dyn_smem(size_t bytes) {
+    if (bytes <= 48 * 1024) return true;
+    static std::atomic<int> done[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+    if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
+    if (cudaFuncSetAttribute(reinterpret_cast<const void*>(kernel), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(bytes)) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
+    return true;
 }
 
 // Persistent grid: enough CTAs to fill every SM at full occupancy, never more than the work.
@@ -121,8 +144,10 @@ nvfp4_status launch_quant(const nvfp4::QuantParams& p, cudaStream_t stream) {
     if (grouped) {
         // CTAs work inside one group at a time, with the group's scale table in shared memory
         constexpr auto kernel = nvfp4::quantize_grouped_kernel<FOUR, RULE, FQ>;
-        const dim3 grid = grouped_grid(static_cast<int64_t>(sm_count()) * ctas_per_sm<kernel>(), p.groups, bpg);
-        kernel<<<grid, kThreads, 0, stream>>>(p);
+        constexpr size_t dyn = quant_dyn_smem<FOUR, FQ>();
+        if (!allow_dyn_smem<kernel>(dyn)) return NVFP4_ERR_CUDA;
+        const dim3 grid = grouped_grid(static_cast<int64_t>(sm_count()) * ctas_per_sm<kernel>(dyn), p.groups, bpg);
+        kernel<<<grid, kThreads, dyn, stream>>>(p);
     } else {
         constexpr auto kernel = nvfp4::quantize_kernel<FOUR, RULE, FQ>;
         const unsigned grid = grid_for<kernel>(p.nblocks);
@@ -204,8 +229,10 @@ nvfp4_status dispatch_quant_amax(nvfp4_mode mode, nvfp4_rule rule, const nvfp4::
 template <bool FOUR, int RULE>
 nvfp4_status launch_quant_gemm(const nvfp4::QuantParams& p, cudaStream_t stream) {
     constexpr auto kernel = nvfp4::quantize_grouped_kernel<FOUR, RULE, false, true>;
-    kernel<<<grouped_grid(static_cast<int64_t>(sm_count()) * ctas_per_sm<kernel>(), 1, p.nblocks), kThreads, 0,
-             stream>>>(p);
+    constexpr size_t dyn = quant_dyn_smem<FOUR, false>();
+    if (!allow_dyn_smem<kernel>(dyn)) return NVFP4_ERR_CUDA;
+    kernel<<<grouped_grid(static_cast<int64_t>(sm_count()) * ctas_per_sm<kernel>(dyn), 1, p.nblocks), kThreads,
+             dyn, stream>>>(p);
     return launch_status();
 }
 
