@@ -95,7 +95,7 @@ struct GroupCtx {
     float alpha, beta6, beta4, yl6, yh6, yl4, yh4;
     bool fast;
     uint32_t ident;   // the kernel argument's identity byte selector (e2m1x8_and_decode)
-    uint32_t lane8, dtab;   // decode table (candidate_tab): lane * 8 and the table's shared address
+    uint32_t lane8, dtab;   // decode table (candidate_tab): (lane % 16) * 8 and the table's shared address
 };
 
 template <bool FOUR>
@@ -254,17 +254,18 @@ __device__ __forceinline__ float candidate(const float2 (&x)[8], float r, float 
 }
 
 // Decode table in shared memory (dynamic, kDecodeTableBytes = 64 KiB): for every E2M1 byte e
-// (two codes) the binary32 values of both codes, in 32 copies at e * 256 + lane * 8, so that
-// the 16 lanes of a shared-memory phase each read their own bank pair whatever bytes they look
-// up. One byte permutation forms a lookup's address: the code byte into bits 8-15 and
-// lane * 8 into bits 0-7. The values are the hardware decode's (cvt.rn.f16x2.e2m1x2, widened).
+// (two codes) the binary32 values of both codes, in 16 copies at e * 256 + c * 8 (c < 16), so
+// that the 16 lanes of a shared-memory phase (lane l reads copy l % 16) each read their own
+// bank pair whatever bytes they look up. One byte permutation forms a lookup's address: the
+// code byte into bits 8-15 and (lane % 16) * 8 into bits 0-7; the second half of each 256-byte
+// row is not used. The values are the hardware decode's (cvt.rn.f16x2.e2m1x2, widened).
 constexpr uint32_t kDecodeTableBytes = 65536;
 
 __device__ __forceinline__ void fill_decode_table(float2* dect) {
-    for (uint32_t i = threadIdx.x; i < 8192u; i += blockDim.x) {
+    for (uint32_t i = threadIdx.x; i < 4096u; i += blockDim.x) {
         uint32_t h0, h1, h2, h3;
-        e2m1x8_to_f16x2(i >> 5, h0, h1, h2, h3);
-        dect[i] = f16x2_to_float2(h0);
+        e2m1x8_to_f16x2(i >> 4, h0, h1, h2, h3);
+        dect[(i >> 4) * 32u + (i & 15u)] = f16x2_to_float2(h0);
     }
 }
 

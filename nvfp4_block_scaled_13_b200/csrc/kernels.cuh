@@ -129,7 +129,7 @@ __device__ __forceinline__ void quant_segment(const QuantParams& p, float2* tab,
     uint32_t a0[8], a1[8];
     if (tile < tend) load_tile(xg, tile, lane, bpg, a0, a1);   // in flight while the table is built
     GroupCtx gc = make_group<FOUR>(FRESH ? ld_acquire_f32(p.amax + g) : __ldg(p.amax + g), kSixM, p.ident);
-    gc.lane8 = lane * 8u;
+    gc.lane8 = (lane & 15u) * 8u;
     gc.dtab = dtab;
     __syncthreads();                       // the previous group's table is no longer read
     fill_scale_tables<FOUR>(tab, gc, threadIdx.x);
@@ -176,7 +176,13 @@ __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kerne
     __shared__ float2 tab[256];   // scale tables (fill_scale_tables)
     extern __shared__ __align__(16) float2 dect[];   // decode table (Four Over Six codes): 64 KiB dynamic
     constexpr bool kDec = FOUR && !FQ;
-    if (kDec) fill_decode_table(dect);
+    if (kDec) {
+        // a launch without the table's dynamic shared memory would read past it: do nothing
+        uint32_t dyn;
+        asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+        if (dyn < kDecodeTableBytes) return;
+        fill_decode_table(dect);
+    }
     const uint32_t dtab = kDec ? smem_addr(dect) : 0u;
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t bpg = static_cast<uint32_t>(p.gdiv.bpg);
