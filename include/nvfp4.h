@@ -46,7 +46,8 @@
  *     memory and never synchronizes the host: work is enqueued on `stream` (0 = the legacy
  *     default stream) and completes in stream order. Its only state between calls is a
  *     per-device cache of device attributes (SM count, occupancies, the symbol address below,
- *     the driver's tensor-map encoder) and one static device word per device: the grid-wide
+ *     the driver's tensor-map encoder, which kernels have had their dynamic shared-memory
+ *     limit raised for the 64 KiB decode table) and one static device word per device: the grid-wide
  *     barrier counter of nvfp4_amax_quantize / nvfp4_amax_fakequant calls made without a
  *     workspace.
  *   - Shapes: groups >= 1, rows >= 0, cols >= 0 with cols % 16 == 0. An empty tensor

@@ -229,8 +229,12 @@ def gemm_nvfp4(a_codes, a_scales, a_alpha, b_codes, b_scales, b_alpha, m: int, n
     a stored value is v(code) * E4M3 block scale * FP32 tensor scale). A[m, k] =
     v(code) * f32(scale of block k / 16), exact in binary64; codes are [rows, k/2] bytes with
     element 2j in the low nibble, scales row-major [rows, k/16] E4M3 bytes. The sum over k is
-    a float64 matrix product (exact for the sizes the tests use: every term has at most 7
-    significant bits); the tensor scales multiply once at the end."""
+    a float64 matrix product. It is not exact in general: every term is a multiple of 2^-20
+    (code values are multiples of 1/2, E4M3 scales of 2^-9) with at most 12 significant bits,
+    so the sum is exact only while every partial sum stays below 2^33; beyond that, the usual
+    dot-product bound gives |error| <= k * 2^-53 * sum_k |A[m, k] B[n, k]|, about 2^-41 of
+    sum |terms| at k = 4096, far below the binary32 accumulation bound the tests compare
+    against (k * 2^-24 * sum |terms|). The tensor scales multiply once at the end."""
     v = e2m1_to_f32(np.arange(16)).astype(np.float64)           # the oracle's decodes, as tables
     sv = e4m3_to_f32(np.arange(256)).astype(np.float64)
 
