@@ -388,7 +388,12 @@ def per_config_leg(nv, torch, dev, stream, peak, resident=None):
     input GB/s (2N / t), algorithmic bytes / t against the HBM peak, amax + quantize, and the
     Four Over Six overhead against scale-6 timed in interleaved repetitions on the same tensor.
     Inputs that fit in L2 are timed cold (a 512 MiB write flushes L2 before each launch) and
-    warm (back to back); the 512 KiB workload is timed by CUDA-graph replay of 50 launches."""
+    warm (back to back); the 512 KiB workload is timed by CUDA-graph replay of 50 launches.
+    Cold has two figures. "cold" comes from CUDA graphs of 10 (flush, launch) pairs against
+    graphs of the 10 flushes alone: the difference over 10 is the launch's device time after a
+    flush, free of the host's launch latency. "cold_single" brackets one launch after a flush
+    with two events, and so also holds the gap between the flush's end and the kernel's start
+    (about 6 us for a one-element kernel, measured the same way)."""
     from nvfp4_block_scaled_13_b200 import synth
 
     s = stream.cuda_stream
@@ -443,6 +448,25 @@ def per_config_leg(nv, torch, dev, stream, peak, resident=None):
             b.synchronize()
             return a.elapsed_time(b)
 
+        def graph_cold_ms(fn, pairs=10, rounds=8):
+            ga, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(ga):
+                for _ in range(pairs):
+                    flush.zero_()
+                    fn()
+            with torch.cuda.graph(gb):
+                for _ in range(pairs):
+                    flush.zero_()
+            ga.replay()
+            gb.replay()
+            torch.cuda.synchronize(dev)
+            ta, tb = [], []
+            for i in range(rounds):
+                for gr, tl in ((ga, ta), (gb, tb)) if i % 2 == 0 else ((gb, tb), (ga, ta)):
+                    tl.append(batch_ms(torch, stream, gr.replay, 1))
+            del ga, gb
+            return (statistics.median(ta) - statistics.median(tb)) / pairs
+
         if small:
             per = {}
             for vname, mode, rule in variants:
@@ -459,8 +483,15 @@ def per_config_leg(nv, torch, dev, stream, peak, resident=None):
                 del graph
             res["timing"] = "warm, CUDA-graph replay of 50 launches"
         else:
-            kinds = [("cold", True), ("warm", False)] if fits_l2 else [("", False)]
+            kinds = [("cold_single", True), ("warm", False)] if fits_l2 else [("", False)]
             per = {}
+            if fits_l2:
+                for rep_i in range(2):
+                    for vname, mode, rule in (variants if rep_i % 2 == 0 else variants[::-1]):
+                        per.setdefault(vname + "_cold", []).append(
+                            graph_cold_ms(lambda mode=mode, rule=rule: launch(mode, rule)))
+                for k in list(per):
+                    per[k] = statistics.median(per[k])
             for kind, cold in kinds:
                 t = {v[0]: [] for v in variants}
                 for rep_i in range(14):
@@ -470,7 +501,9 @@ def per_config_leg(nv, torch, dev, stream, peak, resident=None):
                             t[vname].append(dt)
                 for vname in t:
                     per[vname + (f"_{kind}" if kind else "")] = statistics.median(t[vname])
-            res["timing"] = ("L2 flushed before each launch (cold) and back to back (warm)" if fits_l2
+            res["timing"] = ("L2 flushed before each launch: cold = graphs of (flush, launch) pairs minus graphs "
+                             "of the flushes, per launch; cold_single = one launch between two events after a "
+                             "flush; warm = back to back" if fits_l2
                              else "back to back; the input is larger than L2")
         main_v = variants[-1][0]
         suffix = "_cold" if (fits_l2 and not small) else ""

@@ -261,11 +261,23 @@ __device__ __forceinline__ float candidate(const float2 (&x)[8], float r, float 
 // row is not used. The values are the hardware decode's (cvt.rn.f16x2.e2m1x2, widened).
 constexpr uint32_t kDecodeTableBytes = 65536;
 
+// Work item j (0..255) decodes the four rows 4q .. 4q+3 (q = j / 4) with one conversion word
+// and writes copies 4k .. 4k+3 (k = j % 4) of each as two 16-byte stores; odd q writes its two
+// stores in the other order, so the 8 lanes of a 16-byte store phase hit distinct banks.
 __device__ __forceinline__ void fill_decode_table(float2* dect) {
-    for (uint32_t i = threadIdx.x; i < 4096u; i += blockDim.x) {
-        uint32_t h0, h1, h2, h3;
-        e2m1x8_to_f16x2(i >> 4, h0, h1, h2, h3);
-        dect[(i >> 4) * 32u + (i & 15u)] = f16x2_to_float2(h0);
+    float4* t4 = reinterpret_cast<float4*>(dect);   // a row is 16 float4; copies 2i, 2i+1 share one
+    for (uint32_t j = threadIdx.x; j < 256u; j += blockDim.x) {
+        const uint32_t q = j >> 2, k = j & 3u, o = q & 1u;
+        uint32_t h[4];
+        e2m1x8_to_f16x2(0x03020100u + q * 0x04040404u, h[0], h[1], h[2], h[3]);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const float2 v = f16x2_to_float2(h[m]);
+            const float4 vv = make_float4(v.x, v.y, v.x, v.y);
+            float4* row = t4 + (4u * q + m) * 16u + 2u * k;
+            row[o] = vv;
+            row[1u - o] = vv;
+        }
     }
 }
 

@@ -121,13 +121,16 @@ __device__ __forceinline__ void load_tile(const uint16_t* xg, uint32_t tile, uin
 template <bool FOUR, int RULE, bool FQ, bool SWZ, bool FRESH = false, bool DEC = false>
 __device__ __forceinline__ void quant_segment(const QuantParams& p, float2* tab, int64_t g, uint32_t tile,
                                               uint32_t tend, uint32_t stride, uint32_t lane, bool write_tscale,
-                                              uint32_t dtab = 0) {
+                                              uint32_t dtab = 0, float2* dect = nullptr, bool fill_dec = false) {
     constexpr float kSixM = FOUR ? 1536.0f : 2688.0f;   // 6 * 256 or 6 * 448
     const uint32_t bpg = static_cast<uint32_t>(p.gdiv.bpg);
     const int64_t base = g * static_cast<int64_t>(bpg);
     const uint16_t* xg = p.x + base * 16;
     uint32_t a0[8], a1[8];
-    if (tile < tend) load_tile(xg, tile, lane, bpg, a0, a1);   // in flight while the table is built
+    if (tile < tend) load_tile(xg, tile, lane, bpg, a0, a1);   // in flight while the tables are built
+    if constexpr (DEC) {
+        if (fill_dec) fill_decode_table(dect);   // once per CTA; the barrier below publishes it
+    }
     GroupCtx gc = make_group<FOUR>(FRESH ? ld_acquire_f32(p.amax + g) : __ldg(p.amax + g), kSixM, p.ident);
     gc.lane8 = (lane & 15u) * 8u;
     gc.dtab = dtab;
@@ -181,7 +184,6 @@ __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kerne
         uint32_t dyn;
         asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
         if (dyn < kDecodeTableBytes) return;
-        fill_decode_table(dect);
     }
     const uint32_t dtab = kDec ? smem_addr(dect) : 0u;
     const uint32_t lane = threadIdx.x & 31u;
@@ -200,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, FOUR ? 2 : 4) quantize_grouped_kerne
         const uint32_t t0 = static_cast<uint32_t>(t - g * ntiles);
         const uint32_t t1 = static_cast<uint32_t>(min(end - g * ntiles, static_cast<int64_t>(ntiles)));
         quant_segment<FOUR, RULE, FQ, SWZ, false, kDec>(p, tab, g, t0 + first, t1, stride, lane,
-                                                        one ? blockIdx.x == 0 : t0 == 0, dtab);
+                                                        one ? blockIdx.x == 0 : t0 == 0, dtab, dect, t == begin);
         t = g * ntiles + t1;
     }
 }
