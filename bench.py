@@ -634,12 +634,13 @@ def run_ours(args, rank, world, local):
     # the variants alternate batch by batch.
     variants = [("scale6", 0, 2), ("46_maxerr", 1, 0), ("46_mae", 1, 1), ("46_mse", 1, 2)]
     times = {v[0]: [] for v in variants}
-    for rep in range(10):
-        for name, mode, rule in (variants if rep % 2 == 0 else variants[::-1]):
-            dt = batch_ms(torch, stream, lambda: nv.nvfp4_quantize(xd, g, r, c, amax, mode, rule, codes, scales,
-                                                                   tscale, choice, s), OVERHEAD_BATCH)
-            if rep >= 2:
-                times[name].append(dt)
+    with ClockSampler(local) as clocks_overhead:   # the issue-bound 4/6 kernels follow the SM clock
+        for rep in range(10):
+            for name, mode, rule in (variants if rep % 2 == 0 else variants[::-1]):
+                dt = batch_ms(torch, stream, lambda: nv.nvfp4_quantize(xd, g, r, c, amax, mode, rule, codes, scales,
+                                                                       tscale, choice, s), OVERHEAD_BATCH)
+                if rep >= 2:
+                    times[name].append(dt)
     med = {k: statistics.median(v) for k, v in times.items()}
     overhead = {k: round(med[k] / med["scale6"] - 1.0, 4) for k in med if k != "scale6"}
 
@@ -700,8 +701,10 @@ def run_ours(args, rank, world, local):
     # ---- every workload's quantize kernel (N = 1 only) ----
     per_cfg = None
     if world == 1 and not args.no_per_config:
-        per_cfg = per_config_leg(nv, torch, dev, stream, measured_peak()[0],
-                                 resident={WORKLOAD: (x_np, (g, r, c))} if args.rows is None else None)
+        with ClockSampler(local) as clocks_per_config:
+            per_cfg = per_config_leg(nv, torch, dev, stream, measured_peak()[0],
+                                     resident={WORKLOAD: (x_np, (g, r, c))} if args.rows is None else None)
+        per_cfg["clocks"] = clocks_per_config.summary()
 
     # ---- the FP4 tensor-core GEMM (N = 1 only) ----
     gemm = None
@@ -747,7 +750,8 @@ def run_ours(args, rank, world, local):
                 for k, t in (("amax", t_amax), ("quantize", t_quant), ("dequantize", t_deq))
             },
             "quantize_input_GBps": round(2 * n / (t_quant * 1e-3) / GB, 1),
-            "overhead_46_vs_scale6": {"ms": {k: round(v, 4) for k, v in med.items()}, "overhead": overhead},
+            "overhead_46_vs_scale6": {"ms": {k: round(v, 4) for k, v in med.items()}, "overhead": overhead,
+                                      "clocks": clocks_overhead.summary()},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_k, "wall_s": round(wall, 3),
                     "path": "pinned host x -> H2D -> nvfp4_amax -> nvfp4_quantize -> nvfp4_dequantize -> "
